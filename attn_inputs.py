@@ -1,0 +1,112 @@
+"""Seeded synthetic inputs shared by the oracle tests, the CUDA parity tests and
+the benchmark.
+
+This module only draws random numbers and names the workloads; it holds none
+of the attention arithmetic.  Recipe: a torch CPU ``Generator`` seeded per
+case draws float32 standard normals in the order Q, K, V, dO; optional data
+transforms (Q scaled by 2, K shifted by +8) are applied in float32; then each
+tensor is cast (round to nearest even) to the storage dtype.  The oracle and
+the GPU see identical bits.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    dtype: str = "bf16"          # "bf16" or "f32"
+    seed: int = 0
+    q_mul: float = 1.0           # Q pre-multiplied in float32 before the cast
+    k_add: float = 0.0           # constant added to every K element before the cast
+    backward: bool = True
+
+    @property
+    def Nq(self) -> int:
+        return self.N
+
+    @property
+    def Nk(self) -> int:
+        return self.N
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+
+def _c5() -> list:
+    out = []
+    k = 0
+    for d in (64, 128, 256):
+        for n in (512, 2048, 8192):
+            for causal in (True, False):
+                out.append(Workload(f"sweep_d{d}_n{n}_{'causal' if causal else 'full'}",
+                                    32768 // n, 16, 16, n, d, causal, "bf16", 500 + k))
+                k += 1
+    out.append(Workload("sweep_adversarial_kplus8_d128_n2048_causal", 32768 // 2048, 16, 16, 2048, 128,
+                        True, "bf16", 500 + k, k_add=8.0))
+    return out
+
+
+# The five workloads, by what they are.
+SINGLE_HEAD_F32 = Workload("single_head_f32_n256_d64", 1, 1, 1, 256, 64, False, "f32", 1)
+TWO_BATCH_F32 = Workload("two_batch_f32_n1024_d64", 2, 1, 1, 1024, 64, False, "f32", 2, backward=False)
+TWO_BATCH_BF16 = Workload("two_batch_bf16_n1024_d64", 2, 1, 1, 1024, 64, False, "bf16", 2, backward=False)
+CAUSAL_TRAIN = Workload("causal_b4_h16_n4096_d128", 4, 16, 16, 4096, 128, True, "bf16", 3)
+LONG_GQA = Workload("long_gqa_b1_hq32_hkv8_n16384_d128_q2x", 1, 32, 8, 16384, 128, True, "bf16", 4, q_mul=2.0)
+SWEEP = _c5()
+
+ALL = [SINGLE_HEAD_F32, TWO_BATCH_F32, TWO_BATCH_BF16, CAUSAL_TRAIN, LONG_GQA] + SWEEP
+BY_NAME = {w.name: w for w in ALL}
+
+
+def make(w: Workload, *, B=None, Hq=None, Hkv=None, N=None, Nq=None, Nk=None, d=None,
+         seed=None, dtype=None, q_mul=None, k_add=None):
+    """Draw Q, K, V, dO for workload ``w`` (optionally with shapes overridden).
+
+    Returns a dict of contiguous CPU tensors in the storage dtype:
+    q, do: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]."""
+    B = w.B if B is None else B
+    Hq = w.Hq if Hq is None else Hq
+    Hkv = w.Hkv if Hkv is None else Hkv
+    N = w.N if N is None else N
+    Nq = N if Nq is None else Nq
+    Nk = N if Nk is None else Nk
+    d = w.d if d is None else d
+    seed = w.seed if seed is None else seed
+    dt = w.torch_dtype if dtype is None else (torch.bfloat16 if dtype == "bf16" else torch.float32)
+    q_mul = w.q_mul if q_mul is None else q_mul
+    k_add = w.k_add if k_add is None else k_add
+    return draw(B, Hq, Hkv, Nq, Nk, d, seed, dt, q_mul, k_add)
+
+
+def draw(B, Hq, Hkv, Nq, Nk, d, seed, dtype=torch.bfloat16, q_mul=1.0, k_add=0.0):
+    g = torch.Generator().manual_seed(int(seed))
+    q = torch.randn(B, Hq, Nq, d, generator=g, dtype=torch.float32)
+    k = torch.randn(B, Hkv, Nk, d, generator=g, dtype=torch.float32)
+    v = torch.randn(B, Hkv, Nk, d, generator=g, dtype=torch.float32)
+    do = torch.randn(B, Hq, Nq, d, generator=g, dtype=torch.float32)
+    if q_mul != 1.0:
+        q = q * q_mul
+    if k_add != 0.0:
+        k = k + k_add
+    return {name: t.to(dtype).contiguous() for name, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+
+
+def as_f64(t):
+    """Exact float64 numpy copy of a float32/bf16 tensor."""
+    return t.detach().to("cpu").to(torch.float64).numpy()

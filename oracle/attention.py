@@ -1,0 +1,282 @@
+"""Float64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` call it.  It shares no code with the CUDA library.
+
+What it computes (the plain definition, materialised, in float64):
+
+* Forward -- "FlashAttention" blog (ruizhehou.github.io), section 1 (standard
+  attention): S = Q K^T / sqrt(d), P = softmax(S), O = P V, with the
+  max-subtracted ("safe") softmax of section 2.2.  The CSDN FlashAttention-1
+  tutorial, section 1, gives the same formula softmax(Q K^T / sqrt(d_k)) V.
+  The scale is a parameter (1/sqrt(d) in every workload); the causal mask is
+  the ``is_causal=True`` option of ``F.scaled_dot_product_attention`` quoted
+  in the blog's section 5 (top-left aligned: key j is masked for query i when
+  j > i).
+* Saved statistic -- the blog's section 2.3 keeps m and l per row; this oracle
+  returns the single per-row log-sum-exp L = m + ln(l) of the scaled scores,
+  natural log.
+* Backward -- the pages only say that P is recomputed from Q, K and the saved
+  statistics (blog section 2.3).  The gradients below are the calculus of the
+  forward definition for the scalar f = sum(O * dO):
+      dV = P^T dO,  dP = dO V^T,  D_i = sum_j P_ij dP_ij (= sum_d dO_id O_id),
+      dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q.
+  Pinned by central finite differences and a library cross-check in tests.
+* Grouped-query attention (GQA, named in the wiki's FlashAttention-2 history):
+  query head h reads key/value head floor(h / g), g = Hq / Hkv; dK and dV of a
+  key/value head sum over the g query heads of its group.
+* Block-wise forms -- the online-softmax step of blog section 2.2 (normalise at
+  every block, "v1") and the deferred-normalisation loop of blog section 4.1
+  and the CSDN tutorial section 3 ("v2": keep O unnormalised, rescale by
+  exp(m_old - m_new), divide by l once).  They exist so tests can show the
+  recurrences equal the one-shot softmax; they are never the reference values.
+
+Parity: every function here is pinned by tests/test_oracle.py (closed forms,
+invariants, finite differences, torch float64 SDPA cross-check, a hand-worked
+golden fixture).  No function is "parity unpinned".
+
+Layout: dense [B, H, N, d] arrays (d fastest), any float dtype on input; all
+arithmetic in float64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "scores",
+    "probs",
+    "forward",
+    "backward",
+    "forward_rows",
+    "lse_rows",
+    "backward_rows",
+    "backward_kv_rows",
+    "blockwise_forward_v1",
+    "blockwise_forward_v2",
+]
+
+
+def _f64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def _kv_head(h: int, hq: int, hkv: int) -> int:
+    """GQA mapping: query head h reads key/value head floor(h / g)."""
+    if hq % hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return h // (hq // hkv)
+
+
+def _causal_mask(nq: int, nk: int) -> np.ndarray:
+    """True where key j is hidden from query i (j > i, top-left alignment)."""
+    i = np.arange(nq)[:, None]
+    j = np.arange(nk)[None, :]
+    return j > i
+
+
+def scores(q2, k2, scale, causal):
+    """Masked scaled scores S = scale * q k^T for one head; masked entries -inf.
+
+    Standard attention, blog section 1; causal mask per blog section 5."""
+    s = scale * (_f64(q2) @ _f64(k2).T)
+    if causal:
+        s = np.where(_causal_mask(s.shape[0], s.shape[1]), -np.inf, s)
+    return s
+
+
+def probs(q2, k2, scale, causal):
+    """P = softmax(S) row-wise, max-subtracted (blog section 2.2)."""
+    s = scores(q2, k2, scale, causal)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=1, keepdims=True)
+
+
+def _head_forward(q2, k2, v2, scale, causal):
+    s = scores(q2, k2, scale, causal)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = np.sum(e, axis=1, keepdims=True)
+    p = e / l
+    o = p @ _f64(v2)
+    lse = (m + np.log(l))[:, 0]
+    return o, lse, p
+
+
+def forward(q, k, v, scale, causal):
+    """O = softmax(scale * Q K^T [+ causal mask]) V and L = logsumexp per row.
+
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d].  Returns (o [B,Hq,Nq,d],
+    lse [B,Hq,Nq]) in float64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    Hkv = k.shape[1]
+    o = np.empty((B, Hq, Nq, v.shape[3]))
+    lse = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            kh = _kv_head(h, Hq, Hkv)
+            o[b, h], lse[b, h], _ = _head_forward(q[b, h], k[b, kh], v[b, kh], scale, causal)
+    return o, lse
+
+
+def backward(q, k, v, do, scale, causal):
+    """Gradients of f = sum(O * dO) with respect to Q, K, V.
+
+    P is rebuilt from the definition (not taken from the caller).  Returns
+    (dq, dk, dv, D) with D = rowsum(P * dP) [B, Hq, Nq]."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Hq, Nq, d = q.shape
+    Hkv = k.shape[1]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dsum = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            kh = _kv_head(h, Hq, Hkv)
+            _, _, p = _head_forward(q[b, h], k[b, kh], v[b, kh], scale, causal)
+            dp = do[b, h] @ v[b, kh].T
+            D = np.sum(p * dp, axis=1)
+            ds = p * (dp - D[:, None])
+            dq[b, h] = scale * (ds @ k[b, kh])
+            dk[b, kh] += scale * (ds.T @ q[b, h])
+            dv[b, kh] += p.T @ do[b, h]
+            dsum[b, h] = D
+    return dq, dk, dv, dsum
+
+
+# ---------------------------------------------------------------------------
+# Row-subset forms for full-size workloads.  Attention rows are independent
+# (row i of O and L depends on q_i and all of K, V only), so these are the
+# same definition restricted to chosen rows / columns, evaluated in row chunks
+# so an N x N matrix never has to exist at once.
+# ---------------------------------------------------------------------------
+
+def _row_chunk_scores(q2, k2, scale, causal, rows):
+    s = scale * (_f64(q2)[rows] @ _f64(k2).T)
+    if causal:
+        s = np.where(np.arange(k2.shape[0])[None, :] > np.asarray(rows)[:, None], -np.inf, s)
+    return s
+
+
+def forward_rows(q2, k2, v2, scale, causal, rows):
+    """O and L for the given query rows of one head (q2 [Nq,d], k2/v2 [Nk,d])."""
+    rows = np.asarray(rows)
+    s = _row_chunk_scores(q2, k2, scale, causal, rows)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = np.sum(e, axis=1, keepdims=True)
+    return (e / l) @ _f64(v2), (m + np.log(l))[:, 0]
+
+
+def lse_rows(q2, k2, scale, causal, rows, chunk=2048):
+    """L for the given rows, evaluated chunk by chunk."""
+    rows = np.asarray(rows)
+    out = np.empty(len(rows))
+    for c in range(0, len(rows), chunk):
+        r = rows[c:c + chunk]
+        s = _row_chunk_scores(q2, k2, scale, causal, r)
+        m = np.max(s, axis=1, keepdims=True)
+        out[c:c + chunk] = (m + np.log(np.sum(np.exp(s - m), axis=1, keepdims=True)))[:, 0]
+    return out
+
+
+def backward_rows(q2, k2, v2, do2, scale, causal, rows):
+    """dQ for the given query rows of one head.
+
+    Row i of dS = P_i * (dP_i - D_i) needs only row i of P and dP, so dQ_i is
+    local to the row.  Returns (dq_rows, D_rows)."""
+    rows = np.asarray(rows)
+    s = _row_chunk_scores(q2, k2, scale, causal, rows)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    p = e / np.sum(e, axis=1, keepdims=True)
+    dp = _f64(do2)[rows] @ _f64(v2).T
+    D = np.sum(p * dp, axis=1)
+    ds = p * (dp - D[:, None])
+    return scale * (ds @ _f64(k2)), D
+
+
+def backward_kv_rows(q_heads, k2, v2, do_heads, scale, causal, kv_rows, chunk=2048):
+    """dK and dV for chosen key/value rows of one key/value head.
+
+    q_heads, do_heads: lists of the [Nq, d] query / output-gradient matrices of
+    the g query heads that read this key/value head.  Column j of P needs L_i
+    and D_i of every query row; both are per-row quantities computed here from
+    full rows, chunk by chunk.  Returns (dk_rows, dv_rows) summed over the
+    group."""
+    kv_rows = np.asarray(kv_rows)
+    k2, v2 = _f64(k2), _f64(v2)
+    dk = np.zeros((len(kv_rows), k2.shape[1]))
+    dv = np.zeros((len(kv_rows), v2.shape[1]))
+    for q2, do2 in zip(q_heads, do_heads):
+        q2, do2 = _f64(q2), _f64(do2)
+        nq = q2.shape[0]
+        for c in range(0, nq, chunk):
+            r = np.arange(c, min(c + chunk, nq))
+            s = _row_chunk_scores(q2, k2, scale, causal, r)
+            m = np.max(s, axis=1, keepdims=True)
+            e = np.exp(s - m)
+            p = e / np.sum(e, axis=1, keepdims=True)
+            dp = do2[r] @ v2.T
+            D = np.sum(p * dp, axis=1)
+            pj = p[:, kv_rows]                      # [rows, J]
+            dsj = pj * (dp[:, kv_rows] - D[:, None])
+            dv += pj.T @ do2[r]
+            dk += scale * (dsj.T @ q2[r])
+    return dk, dv
+
+
+# ---------------------------------------------------------------------------
+# Block-wise recurrences (self-checks only).
+# ---------------------------------------------------------------------------
+
+def blockwise_forward_v1(q2, k2, v2, scale, causal, block):
+    """Online softmax that renormalises O at every key block (blog section 2.2:
+    O_new = (e^{m_prev - m_new} l_prev O_prev + e^{S - m_new} V) / l_new)."""
+    q2, k2, v2 = _f64(q2), _f64(k2), _f64(v2)
+    nq, nk = q2.shape[0], k2.shape[0]
+    o = np.zeros((nq, v2.shape[1]))
+    l = np.zeros((nq, 1))
+    m = np.full((nq, 1), -np.inf)
+    for j0 in range(0, nk, block):
+        j1 = min(j0 + block, nk)
+        s = scale * (q2 @ k2[j0:j1].T)
+        if causal:
+            s = np.where(np.arange(j0, j1)[None, :] > np.arange(nq)[:, None], -np.inf, s)
+        m_new = np.maximum(m, np.max(s, axis=1, keepdims=True))
+        # rows whose every key so far is masked keep m = -inf; guard the
+        # factor e^{(-inf) - (-inf)} to 0 (nothing accumulated yet)
+        alpha = np.where(np.isneginf(m_new), 0.0, np.exp(m - np.where(np.isneginf(m_new), 0.0, m_new)))
+        e = np.where(np.isneginf(s), 0.0, np.exp(s - np.where(np.isneginf(m_new), 0.0, m_new)))
+        l_new = alpha * l + np.sum(e, axis=1, keepdims=True)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            o = np.where(l_new > 0, (alpha * l * o + e @ v2[j0:j1]) / np.where(l_new > 0, l_new, 1.0), 0.0)
+        m, l = m_new, l_new
+    return o, (m + np.log(l))[:, 0]
+
+
+def blockwise_forward_v2(q2, k2, v2, scale, causal, block):
+    """Deferred normalisation (blog section 4.1 "v2"; CSDN tutorial section 3):
+    O~ <- e^{m - m_new} O~ + e^{S - m_new} V,  l <- e^{m - m_new} l + rowsum,
+    and one final O = O~ / l."""
+    q2, k2, v2 = _f64(q2), _f64(k2), _f64(v2)
+    nq, nk = q2.shape[0], k2.shape[0]
+    o_t = np.zeros((nq, v2.shape[1]))
+    l = np.zeros((nq, 1))
+    m = np.full((nq, 1), -np.inf)
+    for j0 in range(0, nk, block):
+        j1 = min(j0 + block, nk)
+        s = scale * (q2 @ k2[j0:j1].T)
+        if causal:
+            s = np.where(np.arange(j0, j1)[None, :] > np.arange(nq)[:, None], -np.inf, s)
+        m_new = np.maximum(m, np.max(s, axis=1, keepdims=True))
+        safe = np.where(np.isneginf(m_new), 0.0, m_new)
+        alpha = np.where(np.isneginf(m_new), 0.0, np.exp(m - safe))
+        e = np.where(np.isneginf(s), 0.0, np.exp(s - safe))
+        o_t = alpha * o_t + e @ v2[j0:j1]
+        l = alpha * l + np.sum(e, axis=1, keepdims=True)
+        m = m_new
+    return o_t / l, (m + np.log(l))[:, 0]
