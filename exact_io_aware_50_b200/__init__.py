@@ -1,0 +1,11 @@
+"""Exact scaled-dot-product attention for B200 (sm_100a).
+
+The compute lives in ``libfa.so`` (hand-written CUDA, C ABI in include/fa.h);
+``binding`` marshals arguments to it.  Importing the package does not load
+the library; the first call does, and fails loudly when it is missing.
+"""
+from .binding import (  # noqa: F401
+    FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_ARCH, FA_ERR_CUDA,
+    FA_ERR_TIMEOUT, FaError, lib, lib_path, fa_fwd, fa_bwd, fa_fwd_f32, fa_bwd_f32,
+    fa_bwd_workspace_size, fa_device_status, fa_wait_selftest, fa_strerror, forward, backward,
+)

@@ -1,0 +1,160 @@
+"""ctypes binding of libfa.so -- argument marshalling only.
+
+The ``fa_*`` functions mirror the C ABI one to one (raw device pointers as
+ints, sizes, a CUDA stream handle) and return the status code.  ``forward``
+and ``backward`` take torch CUDA tensors, allocate outputs/workspace with
+torch (device memory only), pass pointers and torch's current stream, and
+raise ``FaError`` on a non-zero status.  Every step of the computation runs in
+the library's CUDA kernels; there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_ALIGNMENT = 3
+FA_ERR_ARCH = 4
+FA_ERR_CUDA = 5
+FA_ERR_TIMEOUT = 6
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libfa.so")
+_lib = None
+
+EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_f32", "fa_bwd_f32",
+           "fa_device_status", "fa_wait_selftest", "fa_strerror")
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({fa_strerror(status)})")
+
+
+def lib():
+    """Load libfa.so (once).  Raises if the built library is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise RuntimeError(f"{lib_path} is missing: build it with "
+                               "`python -m exact_io_aware_50_b200.build`")
+        L = ctypes.CDLL(lib_path)
+        P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        dims = [I, I, I, I, I, I, F, I, P]
+        L.fa_fwd.argtypes = [P] * 5 + dims
+        L.fa_fwd.restype = I
+        L.fa_fwd_f32.argtypes = [P] * 5 + dims
+        L.fa_fwd_f32.restype = I
+        L.fa_bwd.argtypes = [P] * 10 + dims
+        L.fa_bwd.restype = I
+        L.fa_bwd_f32.argtypes = [P] * 10 + dims
+        L.fa_bwd_f32.restype = I
+        L.fa_bwd_workspace_size.argtypes = [I, I, I, I]
+        L.fa_bwd_workspace_size.restype = S
+        L.fa_device_status.argtypes = [P]
+        L.fa_device_status.restype = I
+        L.fa_wait_selftest.argtypes = [ctypes.c_longlong, P]
+        L.fa_wait_selftest.restype = I
+        L.fa_strerror.argtypes = [I]
+        L.fa_strerror.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+# ----------------------------------------------------------------- raw ABI
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
+    return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, int(causal), stream)
+
+
+def fa_fwd_f32(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
+    return lib().fa_fwd_f32(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, int(causal), stream)
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
+    return lib().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale,
+                        int(causal), stream)
+
+
+def fa_bwd_f32(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+               stream=0):
+    return lib().fa_bwd_f32(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale,
+                            int(causal), stream)
+
+
+def fa_bwd_workspace_size(B, Hq, Nq, d):
+    return int(lib().fa_bwd_workspace_size(B, Hq, Nq, d))
+
+
+def fa_device_status(stream=0):
+    return lib().fa_device_status(stream)
+
+
+def fa_wait_selftest(timeout_ns, stream=0):
+    return lib().fa_wait_selftest(int(timeout_ns), stream)
+
+
+def fa_strerror(status):
+    try:
+        return lib().fa_strerror(int(status)).decode()
+    except RuntimeError:
+        return "library not loaded"
+
+
+# ----------------------------------------------------------- torch helpers
+def _check(status, where):
+    if status != FA_OK:
+        raise FaError(status, where)
+
+
+def _shape(q, k):
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and k shapes disagree")
+    return B, Hq, Hkv, Nq, Nk, d
+
+
+def _stream(t):
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
+    """O, L = attention(q, k, v) for contiguous CUDA tensors [B, H, N, d]
+    (bf16 -> fa_fwd, float32 -> fa_fwd_f32)."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
+    scale = d ** -0.5 if scale is None else float(scale)
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    o = torch.empty_like(q) if out is None else out
+    L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32) if lse is None else lse
+    fn = fa_fwd if q.dtype == torch.bfloat16 else fa_fwd_f32
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("dtype must be bfloat16 or float32")
+    _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), B, Hq, Hkv,
+              Nq, Nk, d, scale, causal, _stream(q)), fn.__name__)
+    return o, L
+
+
+def backward(q, k, v, o, lse, dout, scale=None, causal=False, workspace=None):
+    """dQ, dK, dV for f = sum(O * dout); o and lse from ``forward``."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
+    scale = d ** -0.5 if scale is None else float(scale)
+    for t in (q, k, v, o, lse, dout):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_size(B, Hq, Nq, d), device=q.device,
+                                dtype=torch.uint8)
+    fn = fa_bwd if q.dtype == torch.bfloat16 else fa_bwd_f32
+    _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+              dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+              B, Hq, Hkv, Nq, Nk, d, scale, causal, _stream(q)), fn.__name__)
+    return dq, dk, dv

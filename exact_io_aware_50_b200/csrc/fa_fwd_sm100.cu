@@ -1,0 +1,417 @@
+// fa_fwd_sm100.cu -- BF16 attention forward for sm_100a: TMA-fed shared-memory
+// ring, tcgen05 MMA with TMEM accumulators, one softmax thread per query row.
+//
+// Method (FlashAttention blog, sections 2-4; CSDN FlashAttention-1 tutorial,
+// section 3): Q is cut into 128-row tiles (outer loop, one or two tiles per
+// CTA), K and V into 128-row blocks (inner loop).  For every block:
+//     S = Q K_j^T                     tcgen05, bf16 x bf16 -> f32 in TMEM
+//     m_new = max(m, rowmax(S*scale)) softmax thread of the row
+//     P = exp(S*scale - m)            written back to TMEM as bf16
+//     l = e^{m_old - m} l + rowsum(P)
+//     O~ = e^{m_old - m} O~ + P V_j   tcgen05, P from TMEM, V from SMEM
+// and after the last block O = O~ / l, L = m + ln(l) (deferred
+// normalisation, blog section 4.1).  The rescale of O~ is skipped while the
+// running max has grown by less than 2^8 (in base-2 units): p values then stay
+// below 256 and the final divide uses the same stale m, so the result is the
+// same quantity (the wiki's FlashAttention-4 paragraph lists conditional
+// rescaling; the exactness argument is the deferred-normalisation identity).
+//
+// Warp roles (10 warps, 320 threads, one CTA per SM):
+//   warps 0-3  softmax + epilogue for Q tile 0 (thread = TMEM lane = row)
+//   warps 4-7  softmax + epilogue for Q tile 1 (NT == 2)
+//   warp  8    TMA producer (Q once, then K_j / V_j into STAGES-deep rings)
+//   warp  9    MMA issuer (one elected thread)
+// MMA issue order per block j (two tiles): PV0(j), S0(j+1), PV1(j), S1(j+1):
+// the softmax of one tile overlaps the tensor-core work of the other.
+// tcgen05 ops of one thread complete in issue order, and tcgen05.commit
+// arrives after all earlier ops, so "S_t(j+1) ready" also means "PV_t(j)
+// done": the softmax thread may rescale O~ in TMEM right then.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace fa {
+namespace {
+
+constexpr int BM = 128;                 // query rows per tile (MMA M)
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D_, int NT_, int BN_, int STAGES_>
+struct FwdCfg {
+  static constexpr int D = D_, NT = NT_, BN = BN_, STAGES = STAGES_;
+  static constexpr int DCH = D / 64;                      // 128-byte column chunks
+  static constexpr int Q_CHUNK = BM * 128;                // bytes of one chunk of a Q tile
+  static constexpr int KV_CHUNK = BN * 128;
+  static constexpr int Q_TILE = Q_CHUNK * DCH;
+  static constexpr int KV_TILE = KV_CHUNK * DCH;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NT * Q_TILE;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
+  static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
+  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NT],
+  // p_full[NT], o_full[NT], drain
+  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NT + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem base slot, abort flag
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;       // + alignment slack
+  // TMEM columns
+  static constexpr int TM_S = 0;                          // S_t at t*BN
+  static constexpr int TM_O = NT * BN;                    // O_t at TM_O + t*D
+  static constexpr int TM_COLS_USED = NT * (BN + D);
+  static constexpr int TM_ALLOC = 512;
+  static_assert(TM_COLS_USED <= TM_ALLOC, "TMEM budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(BN == 128, "softmax path assumes 128 columns per block");
+};
+
+struct FwdParams {
+  float *o_lse;      // lse output
+  __nv_bfloat16 *o;  // O output
+  int Hq, Hkv, Nq, Nk, nqb;  // nqb = query blocks (of NT*128 rows) per head
+  int BH;            // B * Hq
+  float scale_log2;  // scale * log2(e)
+  int causal;
+  unsigned *err;
+};
+
+template <class C>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t *bars = (uint64_t *)(smem + C::OFF_BAR);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int B_QFULL = 0;
+  const int B_KFULL = 1, B_KEMPTY = 1 + C::STAGES, B_VFULL = 1 + 2 * C::STAGES,
+            B_VEMPTY = 1 + 3 * C::STAGES;
+  const int B_SFULL = 1 + 4 * C::STAGES, B_PFULL = B_SFULL + C::NT, B_OFULL = B_PFULL + C::NT;
+  const int B_DRAIN = B_OFULL + C::NT;
+  uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
+  volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
+
+  const int warp = warp_id_uniform();
+  const int lane = threadIdx.x & 31;
+
+  // Work unit: heavy query blocks first (causal), then (batch, head).
+  const int unit = blockIdx.x;
+  const int qblk = p.nqb - 1 - unit / p.BH;
+  const int bh = unit % p.BH;
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int bh_kv = b * p.Hkv + h / (p.Hq / p.Hkv);
+  const int q_start = qblk * C::NT * BM;
+  const int nkb_all = (p.Nk + C::BN - 1) / C::BN;
+  const int nkb = p.causal ? min(nkb_all, (q_start + C::NT * BM + C::BN - 1) / C::BN) : nkb_all;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar(B_KFULL + s), 1);
+      mbar_init(bar(B_KEMPTY + s), 1);
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_VEMPTY + s), 1);
+    }
+    for (int t = 0; t < C::NT; ++t) {
+      mbar_init(bar(B_SFULL + t), 1);
+      mbar_init(bar(B_PFULL + t), BM);
+      mbar_init(bar(B_OFULL + t), 1);
+    }
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::TM_ALLOC);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  WaitCtx wc{p.err, abort_flag, kWaitLimitNs};
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    int last_k_phase[C::STAGES], last_v_phase[C::STAGES];
+    for (int s = 0; s < C::STAGES; ++s) last_k_phase[s] = last_v_phase[s] = -1;
+    bool ok = true;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(B_QFULL), C::NT * C::Q_TILE);
+      for (int t = 0; t < C::NT; ++t)
+        for (int c = 0; c < C::DCH; ++c)
+          tma_load_3d(sbase + C::OFF_Q + t * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(B_QFULL),
+                      c * 64, q_start + t * BM, bh);
+    }
+    for (int j = 0; j < nkb && ok; ++j) {
+      const int s = j % C::STAGES;
+      const uint32_t ph = (j / C::STAGES) & 1;
+      ok = warp_wait_one(bar(B_KEMPTY + s), ph ^ 1, wc);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(B_KFULL + s), C::KV_TILE);
+        for (int c = 0; c < C::DCH; ++c)
+          tma_load_3d(sbase + C::OFF_K + s * C::KV_TILE + c * C::KV_CHUNK, &tmK, bar(B_KFULL + s),
+                      c * 64, j * C::BN, bh_kv);
+      }
+      last_k_phase[s] = ph;
+      ok = warp_wait_one(bar(B_VEMPTY + s), ph ^ 1, wc);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(B_VFULL + s), C::KV_TILE);
+        for (int c = 0; c < C::DCH; ++c)
+          tma_load_3d(sbase + C::OFF_V + s * C::KV_TILE + c * C::KV_CHUNK, &tmV, bar(B_VFULL + s),
+                      c * 64, j * C::BN, bh_kv);
+      }
+      last_v_phase[s] = ph;
+    }
+    if (!ok && lane == 0) {
+      // Drain: let every copy this warp issued land before the CTA exits.
+      (void)drain_wait(bar(B_QFULL), 0, p.err, kWaitLimitNs);
+      for (int s = 0; s < C::STAGES; ++s) {
+        if (last_k_phase[s] >= 0) (void)drain_wait(bar(B_KFULL + s), last_k_phase[s], p.err, kWaitLimitNs);
+        if (last_v_phase[s] >= 0) (void)drain_wait(bar(B_VFULL + s), last_v_phase[s], p.err, kWaitLimitNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t IDESC_S = idesc_bf16(BM, C::BN, 0, 0);
+    constexpr uint32_t IDESC_PV = idesc_bf16(BM, C::D, 0, 1);
+    auto issue_S = [&](int t, int s) {
+      const uint32_t qa = sbase + C::OFF_Q + t * C::Q_TILE;
+      const uint32_t kb = sbase + C::OFF_K + s * C::KV_TILE;
+#pragma unroll
+      for (int kk = 0; kk < C::D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
+        const uint32_t offk = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
+        mma_ss(tmem + C::TM_S + t * C::BN, sw128_desc(qa + off, 16, 1024),
+               sw128_desc(kb + offk, 16, 1024), IDESC_S, kk > 0);
+      }
+    };
+    auto issue_PV = [&](int t, int s, bool first) {
+      const uint32_t vb = sbase + C::OFF_V + s * C::KV_TILE;
+      const uint32_t pcol = tmem + C::TM_S + t * C::BN + C::BN / 2;
+#pragma unroll
+      for (int kk = 0; kk < C::BN / 16; ++kk) {
+        mma_ts(tmem + C::TM_O + t * C::D, pcol + kk * 8,
+               sw128_desc(vb + kk * 16 * 128, C::KV_CHUNK, 1024), IDESC_PV, (!first) || kk > 0);
+      }
+    };
+    bool ok = warp_wait_one(bar(B_QFULL), 0, wc);
+    if (ok) ok = warp_wait_one(bar(B_KFULL + 0), 0, wc);
+    if (ok) {
+      tc_fence_after();
+      if (lane == 0) {
+        for (int t = 0; t < C::NT; ++t) {
+          issue_S(t, 0);
+          mma_commit(bar(B_SFULL + t));
+        }
+        mma_commit(bar(B_KEMPTY + 0));
+      }
+      __syncwarp();
+    }
+    for (int j = 0; j < nkb && ok; ++j) {
+      const int s = j % C::STAGES;
+      const uint32_t ph = (j / C::STAGES) & 1;
+      const int s1 = (j + 1) % C::STAGES;
+      const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
+      ok = warp_wait_one(bar(B_VFULL + s), ph, wc);
+      if (!ok) break;
+      for (int t = 0; t < C::NT && ok; ++t) {
+        ok = warp_wait_one(bar(B_PFULL + t), j & 1, wc);
+        if (!ok) break;
+        if (t == 0 && j + 1 < nkb) {
+          ok = warp_wait_one(bar(B_KFULL + s1), ph1, wc);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          issue_PV(t, s, j == 0);
+          if (j + 1 < nkb) {
+            issue_S(t, s1);
+            mma_commit(bar(B_SFULL + t));
+            if (t == C::NT - 1) mma_commit(bar(B_KEMPTY + s1));
+          } else {
+            mma_commit(bar(B_OFULL + t));
+          }
+          if (t == C::NT - 1) mma_commit(bar(B_VEMPTY + s));
+        }
+        __syncwarp();
+      }
+    }
+    if (!ok && lane == 0) {
+      // Drain: every MMA issued so far must finish before TMEM is freed.
+      mma_commit(bar(B_DRAIN));
+      (void)drain_wait(bar(B_DRAIN), 0, p.err, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else if (warp < 4 * C::NT) {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;                  // Q tile of this warpgroup
+    const int r = threadIdx.x & 127;          // row within the tile = TMEM lane
+    const int row = q_start + t * BM + r;     // query row
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::TM_S + t * C::BN;
+    const uint32_t tP = tS + C::BN / 2;
+    const uint32_t tO = tmem + lane_off + C::TM_O + t * C::D;
+    const int row_lo = q_start + t * BM;
+    const int limit_row = p.causal ? min(p.Nk, row + 1) : p.Nk;  // keys [0, limit) visible
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkb; ++j) {
+      ok = warp_wait_all(bar(B_SFULL + t), j & 1, wc);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[C::BN];
+#pragma unroll
+      for (int c = 0; c < C::BN / 32; ++c)
+        tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_wait_ld();
+      float *s = reinterpret_cast<float *>(sr);
+      const int col_lo = j * C::BN;
+      const bool need_mask =
+          (col_lo + C::BN > p.Nk) || (p.causal && col_lo + C::BN - 1 > row_lo);
+      if (need_mask) {
+        const int lim = limit_row - col_lo;
+#pragma unroll
+        for (int c = 0; c < C::BN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < C::BN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_new = fmaxf(m_run, mx * p.scale_log2);
+      bool rescale = false;
+      float alpha = 1.f;
+      if (j == 0) {
+        m_run = m_new;
+      } else if (__any_sync(0xffffffffu, m_new - m_run > kRescaleThreshold)) {
+        rescale = true;
+        alpha = fast_exp2(m_run - m_new);
+        m_run = m_new;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float rowsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < C::BN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = fast_exp2(fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_use));
+          const float p1 = fast_exp2(fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_use));
+          rowsum += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tP + c * 16, pk);
+      }
+      l_run = l_run * alpha + rowsum;
+      if (rescale) {
+#pragma unroll 1
+        for (int c = 0; c < C::D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(tO + c * 32, ov);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL + t));
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok) ok = warp_wait_all(bar(B_OFULL + t), 0, wc);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      const bool live = row < p.Nq;
+      __nv_bfloat16 *orow = p.o + ((size_t)bh * p.Nq + (live ? row : 0)) * C::D;
+#pragma unroll 1
+      for (int c = 0; c < C::D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + c * 32, ov);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
+                              __uint_as_float(ov[2 * e + 1]) * inv_l);
+        if (live) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      if (live) p.o_lse[(size_t)bh * p.Nq + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_ALLOC);
+  }
+}
+
+bool make_map(CUtensorMap *m, const void *base, int rows_per_head, int heads, int d,
+              int box_rows) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows_per_head, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows_per_head * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class C>
+int run_fwd(const AttnArgs &a) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, a.Nq, a.B * a.Hq, C::D, BM) ||
+      !make_map(&mk, a.k, a.Nk, a.B * a.Hkv, C::D, C::BN) ||
+      !make_map(&mv, a.v, a.Nk, a.B * a.Hkv, C::D, C::BN))
+    return 5;
+  FwdParams p;
+  p.o_lse = a.lse;
+  p.o = (__nv_bfloat16 *)a.o;
+  p.Hq = a.Hq; p.Hkv = a.Hkv; p.Nq = a.Nq; p.Nk = a.Nk;
+  p.nqb = (a.Nq + C::NT * BM - 1) / (C::NT * BM);
+  p.BH = a.B * a.Hq;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.causal = a.causal;
+  p.err = a.err;
+  auto kern = fwd_kernel<C>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+      cudaSuccess)
+    return 5;
+  const long long units = (long long)p.nqb * p.BH;
+  if (units > 2147483647LL) return 2;
+  kern<<<(unsigned)units, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : 5;
+}
+
+}  // namespace
+
+int launch_fwd_bf16_sm100(const AttnArgs &a) {
+  switch (a.d) {
+    case 64: return run_fwd<FwdCfg<64, 2, 128, 4>>(a);
+    case 128: return run_fwd<FwdCfg<128, 2, 128, 2>>(a);
+    case 256: return run_fwd<FwdCfg<256, 1, 128, 1>>(a);
+    default: return 2;
+  }
+}
+
+}  // namespace fa

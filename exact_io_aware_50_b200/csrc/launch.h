@@ -1,0 +1,44 @@
+// launch.h -- internal host-side launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+struct AttnArgs {
+  const void *q = nullptr, *k = nullptr, *v = nullptr;
+  const void *o_in = nullptr;   // forward output (backward input)
+  const void *dout = nullptr;
+  void *o = nullptr;            // forward output
+  float *lse = nullptr;         // forward output / backward input
+  void *dq = nullptr, *dk = nullptr, *dv = nullptr;
+  void *ws = nullptr;           // backward workspace: D then dQ accumulator
+  int B = 0, Hq = 0, Hkv = 0, Nq = 0, Nk = 0, d = 0;
+  float scale = 0.f;
+  int causal = 0;
+  cudaStream_t stream = nullptr;
+  unsigned *err = nullptr;      // device error word
+};
+
+// Byte offset of the dQ accumulator inside the workspace.
+inline size_t ws_dq_offset(int B, int Hq, int Nq) {
+  size_t dbytes = (size_t)B * Hq * Nq * sizeof(float);
+  return (dbytes + 255) & ~(size_t)255;
+}
+
+// Status codes use the fa_status numbering of fa.h.
+int launch_fwd_f32(const AttnArgs &a);
+int launch_bwd_f32(const AttnArgs &a);
+int launch_fwd_bf16_sm100(const AttnArgs &a);
+int launch_bwd_bf16_sm100(const AttnArgs &a);
+int launch_wait_selftest(long long timeout_ns, cudaStream_t stream, unsigned *err);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+}  // namespace fa

@@ -1,0 +1,132 @@
+/*
+ * fa.h -- C ABI of the exact-attention library (libfa.so), sm_100a only.
+ *
+ * The operation (FlashAttention blog, ruizhehou.github.io, section 1 and
+ * section 3; CSDN FlashAttention-1 tutorial, section 1):
+ *
+ *     S = scale * Q K^T      (causal: S_ij = -inf for j > i, top-left aligned,
+ *                             the is_causal=True option of the blog's
+ *                             section 5 call)
+ *     P = softmax(S)         row-wise, max-subtracted (blog section 2.2)
+ *     O = P V
+ *     L_i = m_i + ln(l_i)    per-row log-sum-exp of the scaled scores, natural
+ *                            log (the blog's section 2.3 saves m and l per row;
+ *                            this library saves the one number L)
+ *
+ * Forward: the tiled online-softmax recurrence with deferred normalisation
+ * (blog section 4.1, "v2"; CSDN tutorial section 3).  Backward: P is
+ * recomputed from Q, K and L rather than stored (blog section 2.3); the
+ * gradients are those of f = sum(O * dO).
+ *
+ * Layout (every tensor dense, row-major, d fastest):
+ *     q, o, dout, dq : [B, Hq,  Nq, d]
+ *     k, v, dk, dv   : [B, Hkv, Nk, d]
+ *     lse            : [B, Hq,  Nq] float32
+ * Grouped-query attention (wiki "FlashAttention", FlashAttention-2 history):
+ * query head h reads key/value head h / (Hq / Hkv); dk and dv of a key/value
+ * head are the sums over its query heads.
+ *
+ * Ownership: the caller allocates every buffer (inputs, outputs, workspace)
+ * in device memory.  Inputs are read only; outputs are fully overwritten.
+ * The library allocates nothing, keeps no per-call state and never
+ * synchronises the host with the device: work is enqueued on `stream` and
+ * the call returns.  Asynchronous execution errors surface at the caller's
+ * next synchronisation, as for any CUDA call.
+ *
+ * Errors: every entry point returns an fa_status; nothing is printed, thrown
+ * or aborted.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *fa_stream_t;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, size <= 0, Hq % Hkv != 0, scale not finite or <= 0 */
+  FA_ERR_UNSUPPORTED = 2, /* head dim or mask combination this build does not run */
+  FA_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
+  FA_ERR_ARCH = 4,        /* current device is not compute capability 10.0 */
+  FA_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  FA_ERR_TIMEOUT = 6      /* a bounded in-kernel wait expired (reported by fa_device_status) */
+} fa_status;
+
+/*
+ * fa_fwd -- BF16 forward.  q, k, v, o: bfloat16; lse: float32.
+ * d must be 64, 128 or 256.  causal != 0 requires Nq == Nk.
+ * Nq, Nk >= 1 (any length; tails are masked).  scale is applied to Q K^T
+ * before the softmax (1/sqrt(d) for standard attention).
+ * Returns FA_ERR_UNSUPPORTED for other head dims, FA_ERR_ALIGNMENT when a
+ * pointer is not 16-byte aligned.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+           fa_stream_t stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of device workspace fa_bwd and fa_bwd_f32
+ * need: the per-row vector D = rowsum(dO * O) (B*Hq*Nq float32, rounded up
+ * to 256 bytes) followed by a float32 dQ accumulator (B*Hq*Nq*d float32).
+ * Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
+
+/*
+ * fa_bwd -- BF16 backward.  q, k, v, o, dout: bfloat16 (o and lse as written
+ * by fa_fwd for the same inputs); dq, dk, dv: bfloat16 outputs; workspace:
+ * at least fa_bwd_workspace_size(B, Hq, Nq, d) bytes of device memory,
+ * 256-byte aligned, contents ignored on entry and clobbered.
+ * Same size rules as fa_fwd.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+           const void *dout, void *dq, void *dk, void *dv, void *workspace,
+           int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+           fa_stream_t stream);
+
+/*
+ * fa_fwd_f32 / fa_bwd_f32 -- the same operations with float32 q, k, v, o,
+ * dout, dq, dk, dv (FP32 CUDA-core arithmetic; correctness path for float32
+ * inputs).  d must be a multiple of 4 and <= 256.
+ */
+int fa_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
+               int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+               fa_stream_t stream);
+int fa_bwd_f32(const float *q, const float *k, const float *v, const float *o,
+               const float *lse, const float *dout, float *dq, float *dk, float *dv,
+               void *workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+               int causal, fa_stream_t stream);
+
+/*
+ * fa_device_status -- synchronises `stream`, then reads and clears the
+ * library's device error word on the current device.  Returns FA_OK, or
+ * FA_ERR_TIMEOUT when a kernel's bounded wait expired since the last call
+ * (that kernel then returned early and its outputs are undefined), or
+ * FA_ERR_CUDA when the synchronisation itself failed.
+ */
+int fa_device_status(fa_stream_t stream);
+
+/*
+ * fa_wait_selftest -- launches one CTA that waits on a shared-memory barrier
+ * nothing ever arrives at, with the library's bounded wait and a limit of
+ * timeout_ns nanoseconds (1 .. 1e9).  The wait gives up, records
+ * FA_ERR_TIMEOUT in the device error word and the kernel returns normally.
+ * Exists so tests can show the timeout path ends cleanly; follow it with
+ * fa_device_status.
+ */
+int fa_wait_selftest(long long timeout_ns, fa_stream_t stream);
+
+/* fa_strerror -- static description of a status code. */
+const char *fa_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

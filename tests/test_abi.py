@@ -1,0 +1,102 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/fa.h declares, and rejects bad arguments before
+touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import exact_io_aware_50_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_f32", "fa_bwd_f32",
+              "fa_strerror", "fa_device_status", "fa_wait_selftest"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = F.lib()
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", F.lib_path], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r" T (fa_\w+)", out))
+    assert set(declared_functions()) <= exported
+    # nothing but the ABI is exported as a function
+    assert exported == set(declared_functions())
+
+
+def test_strerror_covers_codes():
+    for code in range(0, 7):
+        assert F.fa_strerror(code) not in ("", "unknown status")
+    assert F.fa_strerror(99) == "unknown status"
+
+
+def test_workspace_size():
+    B, H, N, d = 4, 16, 4096, 128
+    dbytes = B * H * N * 4
+    assert F.fa_bwd_workspace_size(B, H, N, d) == ((dbytes + 255) // 256) * 256 + B * H * N * d * 4
+    assert F.fa_bwd_workspace_size(0, 1, 1, 64) == 0
+    assert F.fa_bwd_workspace_size(1, 1, 3, 64) == 256 + 3 * 64 * 4
+
+
+FAKE = 1 << 20  # 16-byte aligned non-null address; never dereferenced (rejected first)
+
+
+@pytest.mark.parametrize("fn", ["fa_fwd", "fa_fwd_f32"])
+def test_forward_argument_errors(fn):
+    f = getattr(F, fn)
+    ok = dict(B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=64, scale=0.125, causal=0)
+
+    def call(ptrs=(FAKE,) * 5, **kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(*ptrs, a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"])
+
+    assert call(ptrs=(0, FAKE, FAKE, FAKE, FAKE)) == F.FA_ERR_INVALID_ARG
+    assert call(B=0) == F.FA_ERR_INVALID_ARG
+    assert call(Nk=-1) == F.FA_ERR_INVALID_ARG
+    assert call(Hq=3, Hkv=2) == F.FA_ERR_INVALID_ARG
+    assert call(scale=0.0) == F.FA_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == F.FA_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == F.FA_ERR_INVALID_ARG
+    assert call(causal=1, Nq=8, Nk=9) == F.FA_ERR_UNSUPPORTED
+    if fn == "fa_fwd":
+        assert call(d=96) == F.FA_ERR_UNSUPPORTED
+        assert call(d=32) == F.FA_ERR_UNSUPPORTED
+    else:
+        assert call(d=260) == F.FA_ERR_UNSUPPORTED
+        assert call(d=6) == F.FA_ERR_UNSUPPORTED
+    assert call(ptrs=(FAKE + 2, FAKE, FAKE, FAKE, FAKE)) == F.FA_ERR_ALIGNMENT
+
+
+@pytest.mark.parametrize("fn", ["fa_bwd", "fa_bwd_f32"])
+def test_backward_argument_errors(fn):
+    f = getattr(F, fn)
+
+    def call(ptrs=(FAKE,) * 10, d=64, Hq=2, Hkv=1):
+        return f(*ptrs, 1, Hq, Hkv, 8, 8, d, 0.125, 0)
+
+    assert call(ptrs=(FAKE,) * 9 + (0,)) == F.FA_ERR_INVALID_ARG
+    assert call(Hq=4, Hkv=3) == F.FA_ERR_INVALID_ARG
+    assert call(d=100 if fn == "fa_bwd" else 300) == F.FA_ERR_UNSUPPORTED
+    assert call(ptrs=(FAKE,) * 9 + (FAKE + 16,)) == F.FA_ERR_ALIGNMENT  # workspace needs 256 B
+    assert call(ptrs=(FAKE,) * 6 + (FAKE + 8,) + (FAKE,) * 3) == F.FA_ERR_ALIGNMENT
+
+
+def test_selftest_rejects_bad_limit():
+    assert F.fa_wait_selftest(0) == F.FA_ERR_INVALID_ARG
+    assert F.fa_wait_selftest(2_000_000_000) == F.FA_ERR_INVALID_ARG

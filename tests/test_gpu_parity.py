@@ -1,0 +1,154 @@
+"""GPU parity: the CUDA library against the float64 oracle, element by element,
+on seeded inputs that span several tiles and ragged tails, plus the edge
+cases of the method (one key, one query, causal diagonal, tails shorter than
+a tile, GQA groups)."""
+import numpy as np
+import pytest
+import torch
+
+import attn_inputs
+import exact_io_aware_50_b200 as F
+import oracle
+from parity import check_grad, check_l, check_o, f64, run_full_check, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    F.lib()
+    yield
+
+
+# ------------------------------------------------------------- wait timeout
+def test_bounded_wait_expires_and_context_survives():
+    assert F.fa_device_status() == F.FA_OK
+    assert F.fa_wait_selftest(2_000_000) == F.FA_OK      # 2 ms limit
+    assert F.fa_device_status() == F.FA_ERR_TIMEOUT       # the wait gave up, kernel returned
+    assert F.fa_device_status() == F.FA_OK                # word cleared
+    x = torch.ones(1024, device="cuda")                   # context still usable
+    assert float(x.sum()) == 1024.0
+
+
+# ------------------------------------------------------------- float32 path
+def test_f32_single_head_workload():
+    w = attn_inputs.SINGLE_HEAD_F32
+    run_full_check(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.causal, "f32", w.seed)
+
+
+def test_f32_two_batch_workload():
+    w = attn_inputs.TWO_BATCH_F32
+    run_full_check(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.causal, "f32", w.seed, backward=False)
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 1, 1, 1, 1, 64, False), (1, 2, 1, 37, 37, 64, True), (2, 4, 2, 70, 45, 32, False),
+    (1, 1, 1, 300, 300, 256, True), (1, 2, 2, 33, 129, 100, False), (1, 3, 1, 65, 65, 4, True),
+])
+def test_f32_small(shape):
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    run_full_check(B, Hq, Hkv, Nq, Nk, d, causal, "f32", seed=11)
+
+
+# ------------------------------------------------------------- bf16 forward
+BF16_SMALL = [
+    # B, Hq, Hkv, Nq, Nk, d, causal
+    (1, 1, 1, 128, 128, 128, False),
+    (1, 1, 1, 256, 256, 128, True),
+    (1, 1, 1, 1, 1, 128, False),
+    (1, 1, 1, 1, 300, 64, False),
+    (1, 2, 1, 17, 17, 64, True),
+    (2, 2, 2, 129, 129, 64, True),
+    (1, 2, 2, 300, 300, 128, True),
+    (1, 4, 2, 1000, 1000, 128, True),
+    (1, 2, 1, 640, 384, 128, False),
+    (1, 1, 1, 200, 1000, 256, False),
+    (2, 2, 1, 513, 513, 256, True),
+    (1, 8, 2, 768, 768, 64, False),
+]
+
+
+@pytest.mark.parametrize("shape", BF16_SMALL, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_forward_small(shape):
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    run_full_check(B, Hq, Hkv, Nq, Nk, d, causal, "bf16", seed=21, backward=False)
+
+
+def test_bf16_forward_two_batch_workload():
+    w = attn_inputs.TWO_BATCH_BF16
+    run_full_check(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.causal, "bf16", w.seed, backward=False)
+
+
+def test_bf16_forward_sharp_and_shifted():
+    # Q x 2 sharpens the softmax; K + 8 stresses the running-max rescale.
+    run_full_check(1, 4, 1, 1024, 1024, 128, True, "bf16", seed=31, q_mul=2.0, backward=False)
+    run_full_check(1, 2, 2, 1024, 1024, 128, True, "bf16", seed=32, k_add=8.0, backward=False)
+    run_full_check(1, 2, 2, 700, 700, 64, False, "bf16", seed=33, k_add=8.0, backward=False)
+
+
+def test_bf16_forward_constant_v_and_zero_q():
+    """Closed forms on the GPU path: constant V rows give O = c, zero Q gives
+    the (prefix) mean of V and L = ln(#visible keys)."""
+    B, H, N, d = 1, 2, 300, 128
+    x = attn_inputs.draw(B, H, H, N, N, d, 41)
+    v = torch.zeros_like(x["v"]) + x["v"][:, :, :1, :]
+    g = to_dev(x)
+    o, _ = F.forward(g["q"], g["k"], v.cuda(), None, True)
+    check_o(f64(o), np.broadcast_to(f64(v[:, :, :1, :]), (B, H, N, d)), "bf16")
+    q0 = torch.zeros_like(g["q"])
+    o, lse = F.forward(q0, g["k"], g["v"], None, False)
+    vm = f64(x["v"]).mean(axis=2, keepdims=True)
+    check_o(f64(o), np.broadcast_to(vm, (B, H, N, d)), "bf16")
+    np.testing.assert_allclose(f64(lse), np.log(N), atol=1e-5)
+
+
+# ------------------------------------------------------------- bf16 backward
+BF16_BWD_SMALL = [
+    (1, 1, 1, 128, 128, 128, False),
+    (1, 1, 1, 256, 256, 128, True),
+    (1, 2, 1, 17, 17, 64, True),
+    (1, 1, 1, 1, 1, 128, False),
+    (2, 2, 2, 129, 129, 64, True),
+    (1, 4, 2, 700, 700, 128, True),
+    (1, 2, 1, 640, 384, 128, False),
+    (1, 2, 2, 333, 333, 256, True),
+    (1, 1, 1, 200, 1000, 256, False),
+    (1, 8, 2, 512, 512, 64, False),
+]
+
+
+@pytest.mark.parametrize("shape", BF16_BWD_SMALL, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_backward_small(shape):
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    run_full_check(B, Hq, Hkv, Nq, Nk, d, causal, "bf16", seed=51)
+
+
+def test_bf16_backward_sharp_and_shifted():
+    run_full_check(1, 4, 1, 1024, 1024, 128, True, "bf16", seed=61, q_mul=2.0)
+    run_full_check(1, 2, 2, 768, 768, 128, True, "bf16", seed=62, k_add=8.0)
+
+
+def test_bf16_backward_single_key_gives_zero_dq_dk():
+    x = attn_inputs.draw(1, 2, 1, 50, 1, 64, 71)
+    g = to_dev(x)
+    o, lse = F.forward(g["q"], g["k"], g["v"], None, False)
+    dq, dk, dv = F.backward(g["q"], g["k"], g["v"], o, lse, g["do"], None, False)
+    assert float(dq.abs().max()) == 0.0 and float(dk.abs().max()) == 0.0
+    ref = f64(x["do"]).sum(axis=(1, 2))
+    check_grad(f64(dv)[:, 0, 0], ref, "bf16", "dV")
+
+
+def test_bf16_backward_repeatable_within_tolerance():
+    """Two runs on the same inputs agree within the gradient tolerance (dQ is
+    accumulated with float32 atomics, so bits may differ between runs)."""
+    x = attn_inputs.draw(1, 4, 4, 1024, 1024, 128, 81)
+    g = to_dev(x)
+    o, lse = F.forward(g["q"], g["k"], g["v"], None, True)
+    r1 = F.backward(g["q"], g["k"], g["v"], o, lse, g["do"], None, True)
+    r2 = F.backward(g["q"], g["k"], g["v"], o, lse, g["do"], None, True)
+    for a, b in zip(r1, r2):
+        rel = float((a.float() - b.float()).norm() / b.float().norm())
+        assert rel < 1e-3
+    assert torch.equal(r1[1], r2[1]) and torch.equal(r1[2], r2[2])  # dK, dV deterministic
