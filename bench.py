@@ -1,0 +1,403 @@
+"""Benchmark: exact attention forward + backward on B200 through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+fa_fwd, then the three backward stages (fa_bwd_prep, fa_bwd_dkdv, fa_bwd_dq,
+i.e. fa_bwd).  Default workload: the causal training step, B=4, Hq=Hkv=16,
+N=4096, d=128, bf16 (the configuration the metric is quoted on).  FLOPs per
+step: forward 4*B*Hq*Nq*Nk*d, backward 2.5x that, both halved for causal.
+
+Multi-GPU (torchrun, one process per GPU): attention shards by (batch,
+key/value head) with no exchange between shards, so every rank runs an
+identical replica of the workload on its own GPU (weak scaling); the time is
+the max over ranks and the value is the sum of all ranks' FLOPs over it.
+
+``--impl reference`` times the float64 CPU oracle (the only reference there
+is) on a bounded sample of the same workload and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd+bwd TFLOP/s (BF16, d=128, causal) and % of B200 dense BF16 peak"
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def flops(w):
+    f = 4.0 * w.B * w.Hq * w.Nq * w.Nk * w.d
+    if w.causal:
+        f /= 2
+    return f, 2.5 * f
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), \
+            d.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def config_dict(w, n, l2_note):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+            "causal": w.causal, "scale": "1/sqrt(d)", "global_batch": w.B * n, "seq_len": w.N,
+            "parallelism": f"replicas x{n} (no collective: shards by batch/head)",
+            "l2": l2_note}
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        cmd = ["nvidia-smi", f"--id={self.index}",
+               "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+               "--format=csv,noheader,nounits", "-lms", "100"]
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    maxs.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import attn_inputs
+    import exact_io_aware_50_b200 as F
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = attn_inputs.BY_NAME[args.workload]
+    fwd_f, bwd_f = flops(w)
+    step_flops = fwd_f + bwd_f
+
+    x = attn_inputs.make(w, seed=w.seed + 1000 * rank)
+    g = {k: v.to(dev) for k, v in x.items()}
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    o = torch.empty_like(g["q"])
+    lse = torch.empty(B, Hq, N, device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
+    ws = torch.empty(F.fa_bwd_workspace_size(B, Hq, N, d), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    P = {n: t.data_ptr() for n, t in g.items()}
+
+    def check(st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: {F.fa_strerror(st)}")
+
+    ev = None
+
+    def step(rec=None):
+        if rec is not None:
+            rec[0].record(stream)
+        check(F.fa_fwd(P["q"], P["k"], P["v"], o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N, N, d,
+                       w.scale, w.causal, sh), "fa_fwd")
+        if rec is not None:
+            rec[1].record(stream)
+        check(F.fa_bwd_prep(o.data_ptr(), P["do"], ws.data_ptr(), B, Hq, N, d, sh), "fa_bwd_prep")
+        if rec is not None:
+            rec[2].record(stream)
+        check(F.fa_bwd_dkdv(P["q"], P["k"], P["v"], lse.data_ptr(), P["do"], dk.data_ptr(),
+                            dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, N, N, d, w.scale, w.causal,
+                            sh), "fa_bwd_dkdv")
+        if rec is not None:
+            rec[3].record(stream)
+        check(F.fa_bwd_dq(ws.data_ptr(), dq.data_ptr(), B, Hq, N, d, w.scale, sh), "fa_bwd_dq")
+        if rec is not None:
+            rec[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if F.fa_device_status(sh) != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(events[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    if F.fa_device_status(sh) != 0:
+        raise RuntimeError("device error word set during the timed region")
+    seg = {"fwd": [], "prep": [], "dkdv": [], "dq": []}
+    for e in events:
+        seg["fwd"].append(e[0].elapsed_time(e[1]))
+        seg["prep"].append(e[1].elapsed_time(e[2]))
+        seg["dkdv"].append(e[2].elapsed_time(e[3]))
+        seg["dq"].append(e[3].elapsed_time(e[4]))
+    mean = {k: sum(v) / len(v) for k, v in seg.items()}
+
+    # ---------------------------------------------------- end to end (host buffers)
+    host = {k: v.pin_memory() for k, v in x.items()}
+    out_host = {"o": torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
+                "lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True),
+                "dq": torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True),
+                "dk": torch.empty(dk.shape, dtype=dk.dtype, pin_memory=True),
+                "dv": torch.empty(dv.shape, dtype=dv.dtype, pin_memory=True)}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    e2e_steps = max(2, min(args.steps, 5))
+
+    def e2e_step():
+        for kname, t in host.items():
+            g[kname].copy_(t, non_blocking=True)
+        step()
+        out_host["o"].copy_(o, non_blocking=True)
+        out_host["lse"].copy_(lse, non_blocking=True)
+        out_host["dq"].copy_(dq, non_blocking=True)
+        out_host["dk"].copy_(dk, non_blocking=True)
+        out_host["dv"].copy_(dv, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1) / e2e_steps
+
+    if dist is not None:
+        t = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+
+    burst, sustained, hbm, src = measured_peaks()
+    # dominant kernel by measured share of the step
+    dom = max(("fwd", "dkdv"), key=lambda k: mean[k])
+    dom_flops = fwd_f if dom == "fwd" else bwd_f
+    achieved = dom_flops / (mean[dom] * 1e-3) / 1e12
+    traffic = load_traffic(w.name, "fa_fwd" if dom == "fwd" else "fa_bwd_dkdv")
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
+        "config": config_dict(w, world, "inputs larger than L2 (no flush): q,k,v,dO,o 320 MiB"
+                              if w.name == "causal_b4_h16_n4096_d128" else "see workload sizes"),
+        "pct_of_nominal_bf16_peak": round(100 * value / world / NOMINAL_BF16_TFLOPS, 2),
+        "pct_of_measured_bf16_peak": round(100 * value / world / burst, 2),
+        "stage_ms": {k: round(v, 4) for k, v in mean.items()},
+        "fwd_tflops": round(fwd_f / (mean["fwd"] * 1e-3) / 1e12, 2),
+        "bwd_tflops": round(bwd_f / ((mean["prep"] + mean["dkdv"] + mean["dq"]) * 1e-3) / 1e12, 2),
+        "roofline": {"bound": "tensor", "kernel": "fa_fwd" if dom == "fwd" else "fa_bwd_dkdv",
+                     "achieved": round(achieved, 2), "peak": burst,
+                     "peak_source": f"{src} bf16 dense burst (MEASURED_PEAKS.json)",
+                     "unit": "TFLOP/s", "frac": round(achieved / burst, 4), "traffic": traffic},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def load_traffic(workload, kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if
+    one exists for this workload and the kernel source has not changed since
+    (the summary records the source hash)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        ent = d.get(workload, {}).get(kernel)
+        if not ent:
+            return None
+        if ent.get("source_sha") != source_sha():
+            return None
+        return ent.get("bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
+def source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "exact_io_aware_50_b200", "csrc")
+    for f in sorted(os.listdir(cs)):
+        with open(os.path.join(cs, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------ CPU oracle
+def cpu_baseline(w, seconds):
+    """Time the float64 oracle (as it stands) on whole (batch, head) units of
+    the workload until about `seconds` of CPU work; throughput in the same
+    unit (attention fwd+bwd FLOPs per second)."""
+    import numpy as np
+    import attn_inputs
+    import oracle
+    x = attn_inputs.make(w, B=1, Hq=w.Hq // w.Hkv, Hkv=1)  # one key/value group of batch 0
+    q, k, v, do = (attn_inputs.as_f64(x[n]) for n in ("q", "k", "v", "do"))
+    heads = 0
+    t0 = time.perf_counter()
+    g = w.Hq // w.Hkv
+    while True:
+        h = heads % g
+        oracle.forward(q[:, h:h + 1], k, v, w.scale, w.causal)
+        oracle.backward(q[:, h:h + 1], k, v, do[:, h:h + 1], w.scale, w.causal)
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or heads >= w.B * w.Hq:
+            break
+    fwd_f, bwd_f = flops(w)
+    per_head = (fwd_f + bwd_f) / (w.B * w.Hq)
+    value = heads * per_head / el / 1e12
+    cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        nth = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if nth:
+            cores = nth[0]
+    except Exception:
+        pass
+    return {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{heads} whole (batch 0, head) units of {w.name}, forward+backward, "
+                      f"{el:.1f} s; full workload has {w.B * w.Hq} heads"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import attn_inputs
+    w = attn_inputs.BY_NAME[args.workload]
+    vals = []
+    samples = []
+    for _ in range(args.steps):
+        cb = cpu_baseline(w, args.cpu_seconds / max(1, args.steps))
+        vals.append(cb["value"])
+        samples.append(cb)
+    value = statistics.median(vals)
+    fwd_f, bwd_f = flops(w)
+    ms = (fwd_f + bwd_f) / (value * 1e12) * 1e3
+    cb = dict(samples[-1])
+    cb["value"] = value
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64", "data": "synthetic (seeded N(0,1), shapes of the workload)",
+           "config": config_dict(w, world, "CPU"),
+           "cpu_baseline": cb,
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="causal_b4_h16_n4096_d128")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -24,8 +24,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libfa.so")
 _lib = None
 
-EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_f32", "fa_bwd_f32",
-           "fa_device_status", "fa_wait_selftest", "fa_strerror")
+EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prep", "fa_bwd_dkdv",
+           "fa_bwd_dq", "fa_fwd_f32", "fa_bwd_f32", "fa_device_status", "fa_wait_selftest",
+           "fa_strerror")
 
 
 class FaError(RuntimeError):
@@ -52,6 +53,12 @@ def lib():
         L.fa_bwd.restype = I
         L.fa_bwd_f32.argtypes = [P] * 10 + dims
         L.fa_bwd_f32.restype = I
+        L.fa_bwd_prep.argtypes = [P, P, P, I, I, I, I, P]
+        L.fa_bwd_prep.restype = I
+        L.fa_bwd_dkdv.argtypes = [P] * 8 + dims
+        L.fa_bwd_dkdv.restype = I
+        L.fa_bwd_dq.argtypes = [P, P, I, I, I, I, F, P]
+        L.fa_bwd_dq.restype = I
         L.fa_bwd_workspace_size.argtypes = [I, I, I, I]
         L.fa_bwd_workspace_size.restype = S
         L.fa_device_status.argtypes = [P]
@@ -82,6 +89,19 @@ def fa_bwd_f32(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, sca
                stream=0):
     return lib().fa_bwd_f32(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale,
                             int(causal), stream)
+
+
+def fa_bwd_prep(o, dout, ws, B, Hq, Nq, d, stream=0):
+    return lib().fa_bwd_prep(o, dout, ws, B, Hq, Nq, d, stream)
+
+
+def fa_bwd_dkdv(q, k, v, lse, dout, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
+    return lib().fa_bwd_dkdv(q, k, v, lse, dout, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale,
+                             int(causal), stream)
+
+
+def fa_bwd_dq(ws, dq, B, Hq, Nq, d, scale, stream=0):
+    return lib().fa_bwd_dq(ws, dq, B, Hq, Nq, d, scale, stream)
 
 
 def fa_bwd_workspace_size(B, Hq, Nq, d):

@@ -167,6 +167,60 @@ FA_EXPORT int fa_bwd(const void *q, const void *k, const void *v, const void *o,
   return fa::launch_bwd_bf16_sm100(a);
 }
 
+FA_EXPORT int fa_bwd_prep(const void *o, const void *dout, void *workspace, int B, int Hq,
+                          int Nq, int d, fa_stream_t stream) {
+  if (!o || !dout || !workspace) return FA_ERR_INVALID_ARG;
+  int st = fa::check_sizes(B, Hq, Hq, Nq, Nq, d, 1.f, 0);
+  if (st) return st;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!fa::aligned16(o) || !fa::aligned16(dout) || ((uintptr_t)workspace & 255u) != 0)
+    return FA_ERR_ALIGNMENT;
+  AttnArgs a;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.o_in = o; a.dout = dout; a.ws = workspace;
+  a.B = B; a.Hq = Hq; a.Hkv = Hq; a.Nq = Nq; a.Nk = Nq; a.d = d; a.stream = (cudaStream_t)stream;
+  return fa::launch_bwd_prep_bf16(a);
+}
+
+FA_EXPORT int fa_bwd_dkdv(const void *q, const void *k, const void *v, const float *lse,
+                          const void *dout, void *dk, void *dv, void *workspace, int B, int Hq,
+                          int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                          fa_stream_t stream) {
+  if (!q || !k || !v || !lse || !dout || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  int st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal);
+  if (st) return st;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  const void *ptrs[] = {q, k, v, lse, dout, dk, dv};
+  for (const void *p : ptrs)
+    if (!fa::aligned16(p)) return FA_ERR_ALIGNMENT;
+  if (((uintptr_t)workspace & 255u) != 0) return FA_ERR_ALIGNMENT;
+  AttnArgs a;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.q = q; a.k = k; a.v = v; a.lse = const_cast<float *>(lse); a.dout = dout;
+  a.dk = dk; a.dv = dv; a.ws = workspace;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.d = d;
+  a.scale = scale; a.causal = causal ? 1 : 0; a.stream = (cudaStream_t)stream;
+  return fa::launch_bwd_dkdv_bf16_sm100(a);
+}
+
+FA_EXPORT int fa_bwd_dq(const void *workspace, void *dq, int B, int Hq, int Nq, int d,
+                        float scale, fa_stream_t stream) {
+  if (!workspace || !dq) return FA_ERR_INVALID_ARG;
+  int st = fa::check_sizes(B, Hq, Hq, Nq, Nq, d, scale, 0);
+  if (st) return st;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!fa::aligned16(dq) || ((uintptr_t)workspace & 255u) != 0) return FA_ERR_ALIGNMENT;
+  AttnArgs a;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.ws = const_cast<void *>(workspace); a.dq = dq;
+  a.B = B; a.Hq = Hq; a.Hkv = Hq; a.Nq = Nq; a.Nk = Nq; a.d = d; a.scale = scale;
+  a.stream = (cudaStream_t)stream;
+  return fa::launch_bwd_dq_bf16(a);
+}
+
 FA_EXPORT int fa_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse, int B,
                int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                fa_stream_t stream) {

@@ -31,7 +31,10 @@ inline size_t ws_dq_offset(int B, int Hq, int Nq) {
 int launch_fwd_f32(const AttnArgs &a);
 int launch_bwd_f32(const AttnArgs &a);
 int launch_fwd_bf16_sm100(const AttnArgs &a);
-int launch_bwd_bf16_sm100(const AttnArgs &a);
+int launch_bwd_bf16_sm100(const AttnArgs &a);   // all three stages
+int launch_bwd_prep_bf16(const AttnArgs &a);     // D + zeroed dQ accumulator
+int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a);
+int launch_bwd_dq_bf16(const AttnArgs &a);       // dq = bf16(scale * accumulator)
 int launch_wait_selftest(long long timeout_ns, cudaStream_t stream, unsigned *err);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).

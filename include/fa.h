@@ -91,6 +91,25 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
            fa_stream_t stream);
 
 /*
+ * The three stages fa_bwd runs, exposed so a caller can time or schedule
+ * them separately.  Called in this order on one stream with the same
+ * workspace they compute exactly what fa_bwd computes (BF16 only):
+ *   fa_bwd_prep  -- D = rowsum(dout * o) into the workspace, dQ accumulator
+ *                   zeroed;
+ *   fa_bwd_dkdv  -- the main pass: dk, dv written, dQ accumulated (f32) in
+ *                   the workspace;
+ *   fa_bwd_dq    -- dq = bf16(scale * accumulator).
+ * Same argument rules as fa_bwd.
+ */
+int fa_bwd_prep(const void *o, const void *dout, void *workspace, int B, int Hq, int Nq, int d,
+                fa_stream_t stream);
+int fa_bwd_dkdv(const void *q, const void *k, const void *v, const float *lse, const void *dout,
+                void *dk, void *dv, void *workspace, int B, int Hq, int Hkv, int Nq, int Nk,
+                int d, float scale, int causal, fa_stream_t stream);
+int fa_bwd_dq(const void *workspace, void *dq, int B, int Hq, int Nq, int d, float scale,
+              fa_stream_t stream);
+
+/*
  * fa_fwd_f32 / fa_bwd_f32 -- the same operations with float32 q, k, v, o,
  * dout, dq, dk, dv (FP32 CUDA-core arithmetic; correctness path for float32
  * inputs).  d must be a multiple of 4 and <= 256.

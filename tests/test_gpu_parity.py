@@ -128,6 +128,8 @@ def test_bf16_backward_small(shape):
 def test_bf16_backward_sharp_and_shifted():
     run_full_check(1, 4, 1, 1024, 1024, 128, True, "bf16", seed=61, q_mul=2.0)
     run_full_check(1, 2, 2, 768, 768, 128, True, "bf16", seed=62, k_add=8.0)
+    run_full_check(1, 2, 1, 300, 300, 64, False, "bf16", seed=63, k_add=8.0)
+    run_full_check(1, 2, 2, 256, 256, 256, True, "bf16", seed=64, q_mul=2.0)
 
 
 def test_bf16_backward_single_key_gives_zero_dq_dk():
@@ -135,7 +137,8 @@ def test_bf16_backward_single_key_gives_zero_dq_dk():
     g = to_dev(x)
     o, lse = F.forward(g["q"], g["k"], g["v"], None, False)
     dq, dk, dv = F.backward(g["q"], g["k"], g["v"], o, lse, g["do"], None, False)
-    assert float(dq.abs().max()) == 0.0 and float(dk.abs().max()) == 0.0
+    # dS is zero in exact arithmetic; only f32 rounding of dP - D remains
+    assert float(dq.abs().max()) < 1e-4 and float(dk.abs().max()) < 1e-4
     ref = f64(x["do"]).sum(axis=(1, 2))
     check_grad(f64(dv)[:, 0, 0], ref, "bf16", "dV")
 
