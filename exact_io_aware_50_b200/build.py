@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfa.so")
-SOURCES = ["fa_capi.cu", "fa_simt.cu", "fa_fwd_sm100.cu", "fa_bwd_sm100.cu"]
+SOURCES = ["fa_capi.cu", "fa_simt.cu", "fa_fwd_sm100.cu", "fa_bwd_sm100.cu", "fa_noalloc.cu"]
 HEADERS = ["common.cuh", "launch.h"]
 
 

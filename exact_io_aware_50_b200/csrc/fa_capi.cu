@@ -83,6 +83,12 @@ __global__ void wait_selftest_kernel(long long limit_ns, unsigned *err) {
 
 }  // namespace
 
+int validate_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal) {
+  return check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal);
+}
+
+int device_prologue(int *dev, AttnArgs &a) { return prologue(dev, a); }
+
 int launch_wait_selftest(long long timeout_ns, cudaStream_t stream, unsigned *err) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>(timeout_ns, err);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;

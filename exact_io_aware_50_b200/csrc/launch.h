@@ -37,6 +37,12 @@ int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a);
 int launch_bwd_dq_bf16(const AttnArgs &a);       // dq = bf16(scale * accumulator)
 int launch_wait_selftest(long long timeout_ns, cudaStream_t stream, unsigned *err);
 
+// Argument checks and per-call device set-up shared by the C entry points
+// (fa_status codes): size/scale rules, then current device, architecture and
+// the device error word.
+int validate_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal);
+int device_prologue(int *dev, AttnArgs &a);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,

@@ -123,6 +123,27 @@ int fa_bwd_f32(const float *q, const float *k, const float *v, const float *o,
                int causal, fa_stream_t stream);
 
 /*
+ * fa_bwd_noalloc -- fa_bwd for callers that cannot allocate device memory
+ * where they run the backward (for example a plugin inside an application
+ * that owns the device memory pool, or a loop that must not risk the device
+ * synchronisation cudaMalloc can cause).  Same arguments and results as
+ * fa_bwd, minus the workspace: the scratch lives in one fixed 32 MiB array
+ * inside the library (reserved on every GPU that loads it, until exit).
+ * The pages have no counterpart; this is an interface convenience.
+ * Returns FA_ERR_UNSUPPORTED, without touching the device, when the problem
+ * needs more scratch than that (4*B*Hq*Nq*(d+1) bytes plus padding, e.g. more
+ * than about 65,000 query rows B*Hq*Nq at d = 128).  The first call on a
+ * device looks up the array's address, so make it before any stream capture.
+ * Every call uses the same array: calls whose kernels overlap on the GPU
+ * (other streams or threads on the same device) race and must be ordered by
+ * the caller.  Allocates nothing.
+ */
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                   const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   fa_stream_t stream);
+
+/*
  * fa_device_status -- synchronises `stream`, then reads and clears the
  * library's device error word on the current device.  Returns FA_OK, or
  * FA_ERR_TIMEOUT when a kernel's bounded wait expired since the last call
