@@ -151,12 +151,13 @@ def run_ours(args, rank, world, local_rank):
                        w.scale, w.causal, sh), "fa_fwd")
         if rec is not None:
             rec[1].record(stream)
-        check(F.fa_bwd_prep(o.data_ptr(), P["do"], ws.data_ptr(), B, Hq, N, d, sh), "fa_bwd_prep")
+        check(F.fa_bwd_prep(P["q"], P["k"], o.data_ptr(), lse.data_ptr(), P["do"], ws.data_ptr(), B,
+                            Hq, Hkv, N, N, d, w.scale, sh), "fa_bwd_prep")
         if rec is not None:
             rec[2].record(stream)
-        check(F.fa_bwd_dkdv(P["q"], P["k"], P["v"], lse.data_ptr(), P["do"], dk.data_ptr(),
-                            dv.data_ptr(), ws.data_ptr(), B, Hq, Hkv, N, N, d, w.scale, w.causal,
-                            sh), "fa_bwd_dkdv")
+        check(F.fa_bwd_dkdv(P["q"], P["k"], P["v"], P["do"], dk.data_ptr(), dv.data_ptr(),
+                            ws.data_ptr(), B, Hq, Hkv, N, N, d, w.scale, w.causal, sh),
+              "fa_bwd_dkdv")
         if rec is not None:
             rec[3].record(stream)
         check(F.fa_bwd_dq(ws.data_ptr(), dq.data_ptr(), B, Hq, N, d, w.scale, sh), "fa_bwd_dq")

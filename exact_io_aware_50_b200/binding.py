@@ -53,9 +53,9 @@ def lib():
         L.fa_bwd.restype = I
         L.fa_bwd_f32.argtypes = [P] * 10 + dims
         L.fa_bwd_f32.restype = I
-        L.fa_bwd_prep.argtypes = [P, P, P, I, I, I, I, P]
+        L.fa_bwd_prep.argtypes = [P] * 6 + [I, I, I, I, I, I, F, P]
         L.fa_bwd_prep.restype = I
-        L.fa_bwd_dkdv.argtypes = [P] * 8 + dims
+        L.fa_bwd_dkdv.argtypes = [P] * 7 + dims
         L.fa_bwd_dkdv.restype = I
         L.fa_bwd_dq.argtypes = [P, P, I, I, I, I, F, P]
         L.fa_bwd_dq.restype = I
@@ -91,12 +91,12 @@ def fa_bwd_f32(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, sca
                             int(causal), stream)
 
 
-def fa_bwd_prep(o, dout, ws, B, Hq, Nq, d, stream=0):
-    return lib().fa_bwd_prep(o, dout, ws, B, Hq, Nq, d, stream)
+def fa_bwd_prep(q, k, o, lse, dout, ws, B, Hq, Hkv, Nq, Nk, d, scale, stream=0):
+    return lib().fa_bwd_prep(q, k, o, lse, dout, ws, B, Hq, Hkv, Nq, Nk, d, scale, stream)
 
 
-def fa_bwd_dkdv(q, k, v, lse, dout, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
-    return lib().fa_bwd_dkdv(q, k, v, lse, dout, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale,
+def fa_bwd_dkdv(q, k, v, dout, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
+    return lib().fa_bwd_dkdv(q, k, v, dout, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale,
                              int(causal), stream)
 
 

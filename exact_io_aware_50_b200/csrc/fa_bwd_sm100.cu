@@ -8,25 +8,40 @@
 //     dV = P^T dO     dP = dO V^T        dS = P * (dP - D)
 //     dK = scale * dS^T Q                dQ = scale * dS K
 //
-// Three launches on the caller's stream:
-//   1. preprocess: D_i = sum_d dO_id O_id (f32) and a zeroed f32 dQ
-//      accumulator, both in the caller's workspace;
-//   2. the dK/dV kernel: one CTA per (batch, key/value head, 128-row key
-//      block); it keeps K_j, V_j in shared memory and dK_j, dV_j in TMEM
-//      for the whole loop over the query heads of its group and their 64-row
-//      query blocks, so dK and dV need no atomics.  Per step (transposed
-//      forms, key rows on the 128 TMEM lanes):
-//          S^T  = K_j Q_i^T          dP^T = V_j dO_i^T     (tcgen05, SMEM x SMEM)
-//          P^T  = exp2(S^T * scale*log2e - L_i*log2e),  dS^T = P^T * (dP^T - D_i)
-//                                                          (one thread per key row)
-//          dV  += P^T dO_i           dK  += dS^T Q_i       (tcgen05, A from TMEM)
-//          dQ_i^T = K_j^T dS^T                             (tcgen05, SMEM x SMEM)
-//      and a readout warpgroup adds dQ_i^T into the f32 accumulator with
-//      float32 reductions.  Two TMEM sets (S^T|dP^T, reused for P^T|dS^T and
-//      dQ^T) let S^T/dP^T of step i+1 run while step i is in the elementwise
-//      stage;
-//   3. convert: dQ = bf16(scale * accumulator).
+// Centring K.  Every row of dS sums to zero (sum_j P_ij dP_ij = D_i and
+// sum_j P_ij = 1), so dQ_i = scale * sum_j dS_ij (k_j - c) for any vector c
+// shared by all key rows of a head; and scale * q_i . k_j = scale * q_i .
+// (k_j - c) + scale * q_i . c, where the last term is constant along a row of
+// S and can be moved into L.  With c = the mean of the head's first key rows
+// rounded to integers, the bf16 rounding of dS is no longer multiplied by the
+// mean of K (the +8-shifted K workload makes that term 8x the rest), and K - c
+// is exact in bf16 whenever k and c are within a factor of two (Sterbenz) and
+// equal to K when c = 0.  So the kernels keep K - c, not K, in shared memory.
+//
+// Launches on the caller's stream:
+//   prep   1. c per (batch, key/value head) into the workspace;
+//          2. per query row: D_i, L2_i = log2e * L_i - scale * log2e * q_i . c,
+//             padded to 64-row blocks, and the zeroed f32 dQ accumulator;
+//   dkdv   one CTA per (batch, key/value head, 128-row key block); K - c and
+//          V stay in shared memory and dK, dV in TMEM for the whole loop over
+//          the query heads of the group and their 64-row query blocks, so dK
+//          and dV need no atomics.  Per step (key rows on the 128 TMEM lanes):
+//              S^T = (K-c) Q_i^T      dP^T = V dO_i^T       (tcgen05, SMEM x SMEM)
+//              P^T = exp2(S^T * scale*log2e - L2_i),  dS^T = P^T * (dP^T - D_i)
+//                                                           (one thread per key row
+//                                                            and 32 query columns)
+//              dV += P^T dO_i         dK += dS^T Q_i        (tcgen05, A from TMEM)
+//              dQ_i^T = (K-c)^T dS^T                        (tcgen05, SMEM x SMEM)
+//          and a readout warpgroup adds dQ_i^T into the f32 accumulator with
+//          float32 reductions.  Two TMEM score sets let S^T/dP^T of step i+1
+//          run while step i is in its elementwise stage; Q_i, dO_i and the
+//          row vectors L2_i, D_i arrive through a ring of TMA copies;
+//   dq     dQ = bf16(scale * accumulator).
+// For d = 256 the dK and dV accumulators alone fill TMEM, so dkdv runs two
+// passes over the same key blocks: dV (S^T, P^T, dV), then dK and dQ.
 #include <math.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "launch.h"
@@ -34,48 +49,45 @@
 namespace fa {
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+// Warp roles: 0-7 elementwise stage (two warpgroups, 32 query columns each),
+// 8-11 dQ readout, 12 TMA producer, 13 MMA issuer.
+constexpr int kThreads = 448;
+constexpr int kReadoutWarp0 = 8;
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kCenterRows = 64;   // rows of K averaged into the centering vector c
+constexpr int kCenterRows = 64;   // key rows averaged into the centring vector c
+constexpr int kRowBlock = 64;     // query rows per step (matches the workspace padding)
 
-// Pass layouts.  kFull: dK, dV and dQ in one pass (d = 64, 128).  For
-// d = 256 the dK and dV accumulators alone fill TMEM, so the work is split
-// into two launches over the same key blocks: kDV (S^T, P^T, dV) and kDKDQ
-// (S^T, dP^T, dS^T, dK, dQ).
 enum Mode { kFull = 0, kDV = 1, kDKDQ = 2 };
 
 template <int D_, int MODE_>
 struct BwdCfg {
   static constexpr int D = D_, MODE = MODE_;
-  static constexpr int BN = 128;       // key rows per CTA (MMA M)
-  static constexpr int BM = 64;        // query rows per step (MMA N)
+  static constexpr int BN = 128;         // key rows per CTA (MMA M)
+  static constexpr int BM = kRowBlock;   // query rows per step (MMA N)
   static constexpr int NSETS = MODE == kDKDQ ? 1 : 2;   // TMEM score sets
-  static constexpr int QS = MODE == kDKDQ ? 1 : 2;      // query-stage ring depth
+  static constexpr int QS = MODE == kDKDQ ? 1 : (MODE == kDV ? 2 : (D == 64 ? 4 : 3));
   static constexpr bool HAS_DP = MODE != kDV;
   static constexpr bool HAS_DV = MODE != kDKDQ;
   static constexpr bool HAS_DK = MODE != kDV;
   static constexpr bool HAS_DQ = MODE != kDV;
-  // dQ uses K - c (c: per-head constant vector); see the kernel comment.
-  static constexpr bool CENTER = MODE == kFull;
-  static constexpr int DCH = D / 64;   // 128-byte column chunks
+  static constexpr int DCH = D / 64;     // 128-byte column chunks
   static constexpr int KV_CHUNK = BN * 128;
   static constexpr int KV_TILE = KV_CHUNK * DCH;
   static constexpr int Q_CHUNK = BM * 128;
   static constexpr int Q_TILE = Q_CHUNK * DCH;
   static constexpr int DS_TILE = BN * BM * 2;  // dS^T, bf16, one 128-byte chunk wide
+  static constexpr int ROWVEC = BM * 4;         // bytes of one 64-row slice of L2 or D
   static_assert(BM == 64, "dS^T buffer is one 64-element swizzle chunk wide");
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_KC = OFF_K + KV_TILE;                       // centred K (CENTER)
-  static constexpr int OFF_V = OFF_KC + (CENTER ? KV_TILE : 0);         // V (HAS_DP); follows KC
+  static constexpr int OFF_V = OFF_K + KV_TILE;   // must directly follow K (d = 64 dQ MMA)
   static constexpr int OFF_Q = OFF_V + (HAS_DP ? KV_TILE : 0);
   static constexpr int OFF_DO = OFF_Q + QS * Q_TILE;
   static constexpr int OFF_DS = OFF_DO + QS * Q_TILE;
-  static constexpr int OFF_LSE = OFF_DS + (HAS_DQ ? NSETS * DS_TILE : 0);  // QS x BM floats
-  static constexpr int OFF_DD = OFF_LSE + QS * BM * 4;                      // QS x BM floats
-  static constexpr int OFF_C = OFF_DD + QS * BM * 4;                        // D floats
-  static constexpr int OFF_BAR = OFF_C + D * 4;
+  static constexpr int OFF_L2 = OFF_DS + (HAS_DQ ? NSETS * DS_TILE : 0);
+  static constexpr int OFF_DD = OFF_L2 + QS * ROWVEC;
+  static constexpr int OFF_BAR = OFF_DD + QS * ROWVEC;
   // kv_full, kc_full, q_full[QS], q_empty[QS], s_full[2], p_full[2],
   // dq_full[2], dq_empty[2], final, drain
   static constexpr int NBAR = 2 + 2 * QS + 8 + 2;
@@ -83,10 +95,12 @@ struct BwdCfg {
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   // TMEM columns.
   //   kFull : dV [0, D), dK [D, 2D), set x at 2D + 128x:
-  //           S^T [0,64) dP^T [64,128); then P^T [0,32) dS^T [32,64) dQ^T [64,128)
-  //   kDV   : dV [0, 256), set x at 256 + 64x: S^T [0,64); then P^T [0,32)
-  //   kDKDQ : dK [0, 256), set at 256: S^T [0,64) dP^T [64,128);
-  //           then dS^T [32,64), dQ^T halves [128,192) and [192,256)
+  //           S^T [0,64) dP^T [64,128); then, for query columns 32w..32w+31
+  //           (warpgroup w), P^T at [32w, 32w+16) and dS^T at [32w+16, 32w+32);
+  //           dQ^T [64,128)
+  //   kDV   : dV [0, 256), set x at 256 + 64x: S^T [0,64); then P^T as above
+  //   kDKDQ : dK [0, 256), set at 256: S^T [0,64) dP^T [64,128); then dS^T
+  //           as above, dQ^T halves [128,192) and [192,256)
   static constexpr int TM_DV = 0;
   static constexpr int TM_DK = MODE == kFull ? D : 0;
   static constexpr int TM_SET0 = MODE == kFull ? 2 * D : D;
@@ -100,31 +114,34 @@ struct BwdCfg {
 };
 
 struct BwdParams {
-  const float *lse;        // [B, Hq, Nq]
-  const float *Dsum;       // [B, Hq, Nq]
+  const float *l2;         // [B*Hq][Npad]
+  const float *dsum;       // [B*Hq][Npad]
+  const float *cvec;       // [B*Hkv][D]
   float *dq_acc;           // [B, Hq, Nq, D]
-  const __nv_bfloat16 *k;  // [B, Hkv, Nk, D] (for the centering vector)
   __nv_bfloat16 *dk, *dv;  // [B, Hkv, Nk, D]
-  int Hq, Hkv, Nq, Nk, nqb, nkb, BHkv;
+  int Hq, Hkv, Nq, Nk, npad, nqb, nkb, BHkv;
   float scale, scale_log2;
   int causal;
   unsigned *err;
 };
 
-// dQ and the mean of K.  Every row of dS sums to zero (sum_j P_ij dP_ij =
-// D_i and sum_j P_ij = 1), so dQ_i = scale * sum_j dS_ij (k_j - c) for any
-// vector c that is the same for all key rows of the head.  With c near the
-// mean of K, the bf16 rounding of dS is no longer multiplied by the mean of
-// K (the +8-shifted K workload makes that term 8x the rest).  c is the f32
-// mean of the head's first min(Nk, 64) key rows, computed identically by
-// every CTA of the head.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                const BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base, kept in the shared address space
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   uint64_t *bars = (uint64_t *)(smem + C::OFF_BAR);
   auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -133,9 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             B_FINAL = B_DQEMPTY + 2, B_DRAIN = B_FINAL + 1;
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
-  float *s_lse = (float *)(smem + C::OFF_LSE);
-  float *s_dd = (float *)(smem + C::OFF_DD);
-  float *s_c = (float *)(smem + C::OFF_C);
+  const float *s_l2 = (const float *)(smem + C::OFF_L2);
+  const float *s_dd = (const float *)(smem + C::OFF_DD);
 
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
@@ -158,14 +174,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_KV), 1);
-    mbar_init(bar(B_KC), 128);
+    mbar_init(bar(B_KC), 256);
     for (int s = 0; s < C::QS; ++s) {
       mbar_init(bar(B_QFULL + s), 1);
       mbar_init(bar(B_QEMPTY + s), 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(B_SFULL + x), 1);
-      mbar_init(bar(B_PFULL + x), 128);
+      mbar_init(bar(B_PFULL + x), 256);
       mbar_init(bar(B_DQFULL + x), 1);
       mbar_init(bar(B_DQEMPTY + x), 128);
     }
@@ -208,25 +224,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = (i / C::QS) & 1;
       ok = warp_wait_one(bar(B_QEMPTY + st), ph ^ 1, wc);
       if (!ok) break;
-      const int h = step_head(i), qb = step_qblk(i);
-      const int bh = b * p.Hq + h;
-      const size_t rowbase = (size_t)bh * p.Nq;
-      for (int c = lane; c < C::BM; c += 32) {
-        const int q = qb * C::BM + c;
-        const bool in = q < p.Nq;
-        s_lse[st * C::BM + c] = in ? p.lse[rowbase + q] * kLog2e : INFINITY;
-        s_dd[st * C::BM + c] = in ? p.Dsum[rowbase + q] : 0.f;
+      if (lane == 0) {
+        const int h = step_head(i), qb = step_qblk(i);
+        const int bh = b * p.Hq + h;
+        const size_t vrow = (size_t)bh * p.npad + (size_t)qb * C::BM;
+        const uint32_t fb = bar(B_QFULL + st);
+        mbar_arrive_expect_tx(fb, 2 * C::Q_TILE + 2 * C::ROWVEC);
+        for (int c = 0; c < C::DCH; ++c) {
+          tma_load_3d(sbase + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, fb, c * 64,
+                      qb * C::BM, bh);
+          tma_load_3d(sbase + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmDO, fb, c * 64,
+                      qb * C::BM, bh);
+        }
+        bulk_load(sbase + C::OFF_L2 + st * C::ROWVEC, p.l2 + vrow, C::ROWVEC, fb);
+        bulk_load(sbase + C::OFF_DD + st * C::ROWVEC, p.dsum + vrow, C::ROWVEC, fb);
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(B_QFULL + st), 2 * C::Q_TILE);
-        for (int c = 0; c < C::DCH; ++c) {
-          tma_load_3d(sbase + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(B_QFULL + st),
-                      c * 64, qb * C::BM, bh);
-          tma_load_3d(sbase + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmDO,
-                      bar(B_QFULL + st), c * 64, qb * C::BM, bh);
-        }
-      }
       last_phase[st] = ph;
     }
     if (!ok && lane == 0) {
@@ -261,7 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    // dV += P^T dO_i and dK += dS^T Q_i (K = 64 query rows, 16 per MMA)
+    // dV += P^T dO_i and dK += dS^T Q_i (K = 64 query rows, 16 per MMA).
+    // Query rows 16 kk .. 16 kk + 15 of P^T / dS^T live in the columns of the
+    // warpgroup that produced them: P^T at 32 w + [0, 16), dS^T at
+    // 32 w + [16, 32), w = kk / 2.
     auto issue_dvdk = [&](int x, int st, bool first) {
       const uint32_t qa = sbase + C::OFF_Q + st * C::Q_TILE;
       const uint32_t da = sbase + C::OFF_DO + st * C::Q_TILE;
@@ -269,33 +285,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (C::HAS_DV) {
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk)
-          mma_ts(tmem + C::TM_DV, set + kk * 8, sw128_desc(da + kk * 2048, C::Q_CHUNK, 1024),
-                 IDESC_KV, (!first) || kk > 0);
+          mma_ts(tmem + C::TM_DV, set + (kk >> 1) * 32 + (kk & 1) * 8,
+                 sw128_desc(da + kk * 2048, C::Q_CHUNK, 1024), IDESC_KV, (!first) || kk > 0);
       }
       if (C::HAS_DK) {
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk)
-          mma_ts(tmem + C::TM_DK, set + 32 + kk * 8, sw128_desc(qa + kk * 2048, C::Q_CHUNK, 1024),
-                 IDESC_KV, (!first) || kk > 0);
+          mma_ts(tmem + C::TM_DK, set + (kk >> 1) * 32 + 16 + (kk & 1) * 8,
+                 sw128_desc(qa + kk * 2048, C::Q_CHUNK, 1024), IDESC_KV, (!first) || kk > 0);
       }
     };
     // dQ_i^T = A^T dS^T with K = 128 key rows (16 per MMA) and M = 128 rows of
-    // A^T: [Kc^T ; V^T] for d = 64 (the V half is unused), Kc^T for d = 128,
-    // and the two 128-row halves of K^T for d = 256.
+    // A^T: [(K-c)^T ; V^T] for d = 64 (the V half is unused), (K-c)^T for
+    // d = 128, and the two 128-row halves of (K-c)^T for d = 256.
     auto issue_dq = [&](int x) {
       const uint32_t set = tmem + C::TM_SET0 + x * C::SET_STRIDE;
       const uint32_t dsb = sbase + C::OFF_DS + x * C::DS_TILE;
-      const uint32_t abase = sbase + (C::CENTER ? C::OFF_KC : C::OFF_K);
 #pragma unroll
       for (int half = 0; half < (C::D == 256 ? 2 : 1); ++half) {
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
           mma_ss(set + C::TM_DQ + half * 64,
-                 sw128_desc(abase + half * 2 * C::KV_CHUNK + kk * 2048, C::KV_CHUNK, 1024),
+                 sw128_desc(sbase + C::OFF_K + half * 2 * C::KV_CHUNK + kk * 2048, C::KV_CHUNK, 1024),
                  sw128_desc(dsb + kk * 2048, C::DS_TILE, 1024), IDESC_DQ, kk > 0);
       }
     };
-    bool ok = warp_wait_one(bar(B_KV), 0, wc);
+    // K - c must be in place before the first MMA reads K
+    bool ok = warp_wait_one(bar(B_KC), 0, wc);
     if (ok && nsteps > 0) {
       ok = warp_wait_one(bar(B_QFULL + 0), 0, wc);
       if (ok) {
@@ -307,7 +323,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
     }
-    if (ok && C::CENTER && nsteps > 0) ok = warp_wait_one(bar(B_KC), 0, wc);
     for (int i = 0; i < nsteps && ok; ++i) {
       const int x = set_of(i);
       const int st = i % C::QS;
@@ -365,48 +380,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------ elementwise stage
-    const int r = threadIdx.x;                     // key row within the block = TMEM lane
+    const int wg = warp >> 2;                      // query columns [32 wg, 32 wg + 32)
+    const int r = threadIdx.x & 127;               // key row within the block = TMEM lane
     const int kv = kv0 + r;
     const bool kv_live = kv < p.Nk;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    bool ok = true;
-    if (C::CENTER) {
-      // c = mean of the head's first rows of K (f32, fixed order)
-      if (r < C::D) {
-        const __nv_bfloat16 *kh = p.k + (size_t)bhkv * p.Nk * C::D + r;
-        const int nr = min(p.Nk, kCenterRows);
-        float acc = 0.f;
-        for (int j = 0; j < nr; ++j) acc += __bfloat162float(kh[(size_t)j * C::D]);
-        s_c[r] = acc / (float)nr;
-      }
-      named_barrier_sync(1, 128);
-      ok = warp_wait_all(bar(B_KV), 0, wc);
-      if (ok) {
-        // Kc row r = bf16(K row r - c) in the same swizzled layout (zero past Nk)
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    // K row r -> K - c in place (same swizzled layout; rows past Nk were
+    // zero-filled and stay zero).  Warpgroup wg takes the 64-column chunks
+    // ch = wg, wg + 2, ...
+    bool ok = warp_wait_all(bar(B_KV), 0, wc);
+    if (ok) {
+      const float *cv = p.cvec + (size_t)bhkv * C::D;
 #pragma unroll 1
-        for (int ch = 0; ch < C::DCH; ++ch) {
-          const uint8_t *src = smem + C::OFF_K + ch * C::KV_CHUNK + r * 128;
-          uint8_t *dst = smem + C::OFF_KC + ch * C::KV_CHUNK + r * 128;
+      for (int ch = wg; ch < C::DCH; ch += 2) {
+        uint8_t *row = smem + C::OFF_K + ch * C::KV_CHUNK + r * 128;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int col = ch * 64 + ((u ^ (r & 7)) << 3);
-            uint4 v = *reinterpret_cast<const uint4 *>(src + (u << 4));
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        for (int u = 0; u < 8; ++u) {
+          const int col = ch * 64 + ((u ^ (r & 7)) << 3);
+          const float4 c_lo = *reinterpret_cast<const float4 *>(cv + col);
+          const float4 c_hi = *reinterpret_cast<const float4 *>(cv + col + 4);
+          const float cc[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
+          uint4 v = *reinterpret_cast<const uint4 *>(row + (u << 4));
+          uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
-              const float2 f = __bfloat1622float2(h2);
-              w[e] = kv_live ? pack_bf16x2(f.x - s_c[col + 2 * e], f.y - s_c[col + 2 * e + 1]) : 0u;
-            }
-            *reinterpret_cast<uint4 *>(dst + (u << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+            const float2 f = __bfloat1622float2(h2);
+            w[e] = kv_live ? pack_bf16x2(f.x - cc[2 * e], f.y - cc[2 * e + 1]) : 0u;
           }
+          *reinterpret_cast<uint4 *>(row + (u << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(bar(B_KC));
       }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_KC));
     }
+    const int c0 = wg * 32;
     for (int i = 0; i < nsteps && ok; ++i) {
       const int x = set_of(i), st = i % C::QS;
       ok = warp_wait_all(bar(B_QFULL + st), (i / C::QS) & 1, wc);
@@ -414,44 +424,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t set = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE;
-      uint32_t sv[64], dv[64];
-      tmem_ld32(set, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(set + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      if (C::HAS_DP) {
-        tmem_ld32(set + 64, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
-        tmem_ld32(set + 96, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
-      }
+      uint32_t sv[32], dv[32];
+      tmem_ld32(set + c0, sv);
+      if (C::HAS_DP) tmem_ld32(set + 64 + c0, dv);
       tmem_wait_ld();
-      const float *lse2 = s_lse + st * C::BM;
-      const float *dd = s_dd + st * C::BM;
-      const int q0 = step_qblk(i) * C::BM;
+      const float4 *l4 = reinterpret_cast<const float4 *>(s_l2 + st * C::BM + c0);
+      const float4 *d4 = reinterpret_cast<const float4 *>(s_dd + st * C::BM + c0);
+      const int q0 = step_qblk(i) * C::BM + c0;
       // causal: key kv is hidden from query q when kv > q; key rows past Nk
-      // (zero-filled) are masked so they add nothing anywhere
-      const int first_vis = !kv_live ? C::BM : (p.causal ? kv - q0 : 0);
-      uint32_t pk[32], dk[32];
+      // (zero-filled) are masked so they add nothing anywhere.  Query rows
+      // past Nq have L2 = +inf, so their P is 0.
+      const int first_vis = !kv_live ? 32 : (p.causal ? kv - q0 : 0);
+      const bool unmasked = __all_sync(0xffffffffu, first_vis <= 0);
+      uint32_t pk[16], dk[16];
+      auto body = [&](auto masked_tag) {
+        constexpr bool MASKED = decltype(masked_tag)::value;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        float pr[2], ds[2];
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 lq = l4[e4];
+          const float4 dq4 = C::HAS_DP ? d4[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
+          const float dvv[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
+          float pr[4], ds[4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = 2 * e + u;
-          float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lse2[c]));
-          pv = (c >= first_vis) ? pv : 0.f;
-          pr[u] = pv;
-          ds[u] = C::HAS_DP ? pv * (__uint_as_float(dv[c]) - dd[c]) : 0.f;
+          for (int u = 0; u < 4; ++u) {
+            const int c = 4 * e4 + u;
+            float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[u]));
+            if (MASKED) pv = (c >= first_vis) ? pv : 0.f;
+            pr[u] = pv;
+            ds[u] = C::HAS_DP ? pv * (__uint_as_float(dv[c]) - dvv[u]) : 0.f;
+          }
+          pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
+          pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
+          dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+          dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        pk[e] = pack_bf16x2(pr[0], pr[1]);
-        dk[e] = pack_bf16x2(ds[0], ds[1]);
-      }
-      if (C::HAS_DV) tmem_st32(set, pk);
-      if (C::HAS_DK) tmem_st32(set + 32, dk);
+      };
+      if (unmasked) body(std::false_type{});
+      else body(std::true_type{});
+      // bf16 P^T and dS^T go into this warpgroup's own (already read) S^T
+      // columns, so the other warpgroup's unread columns are never touched
+      if (C::HAS_DV) tmem_st16(set + c0, pk);
+      if (C::HAS_DK) tmem_st16(set + c0 + 16, dk);
       if (C::HAS_DQ) {
         // dS^T row r -> shared memory (B operand of the dQ^T MMA, 128-byte
-        // swizzled rows: 16-byte chunk c of row r sits at chunk c ^ (r % 8))
+        // swizzled rows: 16-byte chunk c of row r sits at chunk c ^ (r % 8));
+        // this warpgroup owns chunks 4 wg .. 4 wg + 3
         uint8_t *dsrow = smem + C::OFF_DS + x * C::DS_TILE + r * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(dsrow + ((c ^ (r & 7)) << 4)) =
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4 *>(dsrow + (((4 * wg + c) ^ (r & 7)) << 4)) =
               make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
         fence_proxy_async_smem();
       }
@@ -460,44 +482,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_PFULL + x));
     }
     // ------------------------------------------------------ epilogue
+    // warpgroup 0 writes dV, warpgroup 1 writes dK (one key row per thread)
+    const bool mine = wg == 0 ? C::HAS_DV : C::HAS_DK;
     if (ok) ok = warp_wait_all(bar(B_FINAL), 0, wc);
-    if (ok && nsteps > 0) {
+    if (ok && nsteps > 0 && mine) {
       tc_fence_after();
       const size_t rowoff = ((size_t)bhkv * p.Nk + (kv_live ? kv : 0)) * C::D;
+      const uint32_t src = tmem + lane_off + (wg ? C::TM_DK : C::TM_DV);
+      __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + rowoff;
+      const float mul = wg ? p.scale : 1.f;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        if (which == 0 && !C::HAS_DV) continue;
-        if (which == 1 && !C::HAS_DK) continue;
-        const uint32_t src = tmem + lane_off + (which ? C::TM_DK : C::TM_DV);
-        __nv_bfloat16 *dst = (which ? p.dk : p.dv) + rowoff;
-        const float mul = which ? p.scale : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < C::D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(src + c * 32, v);
-          tmem_wait_ld();
-          uint32_t pkd[16];
+      for (int c = 0; c < C::D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(src + c * 32, v);
+        tmem_wait_ld();
+        uint32_t pkd[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pkd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-          if (kv_live) {
-            uint4 *o = reinterpret_cast<uint4 *>(dst + c * 32);
+        for (int e = 0; e < 16; ++e)
+          pkd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+        if (kv_live) {
+          uint4 *o = reinterpret_cast<uint4 *>(dst + c * 32);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) o[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
-          }
+          for (int e = 0; e < 4; ++e) o[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
         }
       }
-    } else if (ok && nsteps == 0 && kv_live) {
+    } else if (ok && nsteps == 0 && kv_live && mine) {
       // no query row sees this key block: its gradients are zero
-      const size_t rowoff = ((size_t)bhkv * p.Nk + kv) * C::D;
-      for (int e = 0; e < C::D / 8; ++e) {
-        if (C::HAS_DK) reinterpret_cast<uint4 *>(p.dk + rowoff)[e] = make_uint4(0, 0, 0, 0);
-        if (C::HAS_DV) reinterpret_cast<uint4 *>(p.dv + rowoff)[e] = make_uint4(0, 0, 0, 0);
-      }
+      __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + ((size_t)bhkv * p.Nk + kv) * C::D;
+      for (int e = 0; e < C::D / 8; ++e) reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0, 0, 0, 0);
     }
-  } else if (warp < 8 && C::HAS_DQ) {
+  } else if (warp < kProducerWarp && C::HAS_DQ) {
     // ------------------------------------------------ dQ readout
-    const int t = threadIdx.x - 128;               // TMEM lane = column d of dQ (per half)
+    const int t = threadIdx.x - 32 * kReadoutWarp0;  // TMEM lane = column d of dQ (per half)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     for (int i = 0; i < nsteps; ++i) {
       const int x = set_of(i);
@@ -536,30 +552,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// D_i = sum_d dO_id * O_id in f32 (one warp per row) and zero the dQ
-// accumulator rows of this warp.
+// c[b, hkv, :] = mean of the head's first min(Nk, 64) key rows, rounded to
+// integers (f32).  One CTA per (batch, key/value head), one thread per column.
 template <int D>
-__global__ void bwd_preprocess_kernel(const __nv_bfloat16 *__restrict__ o,
+__global__ void bwd_center_kernel(const __nv_bfloat16 *__restrict__ k, float *__restrict__ cvec,
+                                  int Nk) {
+  const int t = threadIdx.x;
+  const __nv_bfloat16 *kh = k + (size_t)blockIdx.x * Nk * D + t;
+  const int nr = min(Nk, kCenterRows);
+  float acc = 0.f;
+  for (int j = 0; j < nr; ++j) acc += __bfloat162float(kh[(size_t)j * D]);
+  cvec[(size_t)blockIdx.x * D + t] = rintf(acc / (float)nr);
+}
+
+// Per padded query row (one warp each): D = sum_d dO * O and
+// L2 = log2e * L - scale * log2e * (q . c) (rows past Nq: D = 0, L2 = +inf);
+// zero the row of the dQ accumulator.
+template <int D>
+__global__ void bwd_preprocess_kernel(const __nv_bfloat16 *__restrict__ q,
+                                      const __nv_bfloat16 *__restrict__ o,
                                       const __nv_bfloat16 *__restrict__ dout,
-                                      float *__restrict__ Dsum, float *__restrict__ dq_acc,
-                                      long long rows) {
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+                                      const float *__restrict__ lse,
+                                      const float *__restrict__ cvec, float *__restrict__ dsum,
+                                      float *__restrict__ l2, float *__restrict__ dq_acc,
+                                      long long prow_total, int Nq, int npad, int Hq, int g,
+                                      float scale_log2) {
+  const long long prow = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
+  if (prow >= prow_total) return;
+  const long long bh = prow / npad;
+  const int qi = (int)(prow - bh * npad);
+  if (qi >= Nq) {
+    if (lane == 0) {
+      dsum[prow] = 0.f;
+      l2[prow] = INFINITY;
+    }
+    return;
+  }
+  const long long row = bh * Nq + qi;
+  const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+  const float *cv = cvec + ((size_t)b * (Hq / g) + h / g) * D;
   constexpr int PER = D / 32;  // elements per lane (2, 4 or 8)
-  float s = 0.f;
+  float sd = 0.f, sq = 0.f;
   const __nv_bfloat16 *orow = o + row * D + lane * PER;
   const __nv_bfloat16 *drow = dout + row * D + lane * PER;
+  const __nv_bfloat16 *qrow = q + row * D + lane * PER;
 #pragma unroll
   for (int e = 0; e < PER; e += 2) {
     const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(orow + e));
     const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(drow + e));
-    s = fmaf(a.x, c.x, s);
-    s = fmaf(a.y, c.y, s);
+    const float2 qq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(qrow + e));
+    sd = fmaf(a.x, c.x, sd);
+    sd = fmaf(a.y, c.y, sd);
+    sq = fmaf(qq.x, cv[lane * PER + e], sq);
+    sq = fmaf(qq.y, cv[lane * PER + e + 1], sq);
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) Dsum[row] = s;
+  for (int off = 16; off > 0; off >>= 1) {
+    sd += __shfl_xor_sync(0xffffffffu, sd, off);
+    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+  }
+  if (lane == 0) {
+    dsum[prow] = sd;
+    l2[prow] = lse[row] * kLog2e - scale_log2 * sq;
+  }
   float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D);
   for (int e = lane; e < D / 4; e += 32) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
@@ -592,20 +648,34 @@ bool make_map(CUtensorMap *m, const void *base, int rows_per_head, int heads, in
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+struct WsPtrs {
+  float *dsum, *l2, *cvec, *dq_acc;
+};
+WsPtrs ws_ptrs(const AttnArgs &a) {
+  char *w = (char *)a.ws;
+  return {(float *)w, (float *)(w + ws_l2_offset(a.B, a.Hq, a.Nq)),
+          (float *)(w + ws_c_offset(a.B, a.Hq, a.Nq)),
+          (float *)(w + ws_dq_offset(a.B, a.Hq, a.Nq, a.d))};
+}
+
 template <int D>
 int run_prep(const AttnArgs &a) {
-  float *Dsum = (float *)a.ws;
-  float *dq_acc = (float *)((char *)a.ws + ws_dq_offset(a.B, a.Hq, a.Nq));
-  const long long rows = (long long)a.B * a.Hq * a.Nq;
-  bwd_preprocess_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, a.stream>>>(
-      (const __nv_bfloat16 *)a.o_in, (const __nv_bfloat16 *)a.dout, Dsum, dq_acc, rows);
+  const WsPtrs w = ws_ptrs(a);
+  bwd_center_kernel<D><<<(unsigned)(a.B * a.Hkv), D, 0, a.stream>>>(
+      (const __nv_bfloat16 *)a.k, w.cvec, a.Nk);
+  if (cudaGetLastError() != cudaSuccess) return 5;
+  const int npad = (int)ws_npad(a.Nq);
+  const long long prows = (long long)a.B * a.Hq * npad;
+  bwd_preprocess_kernel<D><<<(unsigned)((prows + 7) / 8), 256, 0, a.stream>>>(
+      (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.o_in, (const __nv_bfloat16 *)a.dout,
+      a.lse, w.cvec, w.dsum, w.l2, w.dq_acc, prows, a.Nq, npad, a.Hq, a.Hq / a.Hkv,
+      a.scale * kLog2e);
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }
 
 template <class C>
 int run_dkdv(const AttnArgs &a) {
-  float *Dsum = (float *)a.ws;
-  float *dq_acc = (float *)((char *)a.ws + ws_dq_offset(a.B, a.Hq, a.Nq));
+  const WsPtrs w = ws_ptrs(a);
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, a.q, a.Nq, a.B * a.Hq, C::D, C::BM) ||
       !make_map(&mdo, a.dout, a.Nq, a.B * a.Hq, C::D, C::BM) ||
@@ -613,13 +683,14 @@ int run_dkdv(const AttnArgs &a) {
       !make_map(&mv, a.v, a.Nk, a.B * a.Hkv, C::D, C::BN))
     return 5;
   BwdParams p;
-  p.lse = a.lse;
-  p.k = (const __nv_bfloat16 *)a.k;
-  p.Dsum = Dsum;
-  p.dq_acc = dq_acc;
+  p.l2 = w.l2;
+  p.dsum = w.dsum;
+  p.cvec = w.cvec;
+  p.dq_acc = w.dq_acc;
   p.dk = (__nv_bfloat16 *)a.dk;
   p.dv = (__nv_bfloat16 *)a.dv;
   p.Hq = a.Hq; p.Hkv = a.Hkv; p.Nq = a.Nq; p.Nk = a.Nk;
+  p.npad = (int)ws_npad(a.Nq);
   p.nqb = (a.Nq + C::BM - 1) / C::BM;
   p.nkb = (a.Nk + C::BN - 1) / C::BN;
   p.BHkv = a.B * a.Hkv;
@@ -638,10 +709,10 @@ int run_dkdv(const AttnArgs &a) {
 }
 
 int run_dq(const AttnArgs &a) {
-  const float *dq_acc = (const float *)((const char *)a.ws + ws_dq_offset(a.B, a.Hq, a.Nq));
+  const WsPtrs w = ws_ptrs(a);
   const long long n8 = (long long)a.B * a.Hq * a.Nq * a.d / 8;
   bwd_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, a.stream>>>(
-      dq_acc, (__nv_bfloat16 *)a.dq, n8, a.scale);
+      w.dq_acc, (__nv_bfloat16 *)a.dq, n8, a.scale);
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }
 

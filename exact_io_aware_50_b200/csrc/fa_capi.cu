@@ -130,7 +130,7 @@ FA_EXPORT const char *fa_strerror(int status) {
 
 FA_EXPORT size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {
   if (B <= 0 || Hq <= 0 || Nq <= 0 || d <= 0) return 0;
-  return fa::ws_dq_offset(B, Hq, Nq) + (size_t)B * Hq * Nq * d * sizeof(float);
+  return fa::ws_bytes(B, Hq, Nq, d);
 }
 
 FA_EXPORT int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
@@ -173,39 +173,41 @@ FA_EXPORT int fa_bwd(const void *q, const void *k, const void *v, const void *o,
   return fa::launch_bwd_bf16_sm100(a);
 }
 
-FA_EXPORT int fa_bwd_prep(const void *o, const void *dout, void *workspace, int B, int Hq,
-                          int Nq, int d, fa_stream_t stream) {
-  if (!o || !dout || !workspace) return FA_ERR_INVALID_ARG;
-  int st = fa::check_sizes(B, Hq, Hq, Nq, Nq, d, 1.f, 0);
+FA_EXPORT int fa_bwd_prep(const void *q, const void *k, const void *o, const float *lse,
+                          const void *dout, void *workspace, int B, int Hq, int Hkv, int Nq,
+                          int Nk, int d, float scale, fa_stream_t stream) {
+  if (!q || !k || !o || !lse || !dout || !workspace) return FA_ERR_INVALID_ARG;
+  int st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, 0);
   if (st) return st;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  if (!fa::aligned16(o) || !fa::aligned16(dout) || ((uintptr_t)workspace & 255u) != 0)
-    return FA_ERR_ALIGNMENT;
-  AttnArgs a;
-  int dev;
-  if ((st = fa::prologue(&dev, a))) return st;
-  a.o_in = o; a.dout = dout; a.ws = workspace;
-  a.B = B; a.Hq = Hq; a.Hkv = Hq; a.Nq = Nq; a.Nk = Nq; a.d = d; a.stream = (cudaStream_t)stream;
-  return fa::launch_bwd_prep_bf16(a);
-}
-
-FA_EXPORT int fa_bwd_dkdv(const void *q, const void *k, const void *v, const float *lse,
-                          const void *dout, void *dk, void *dv, void *workspace, int B, int Hq,
-                          int Hkv, int Nq, int Nk, int d, float scale, int causal,
-                          fa_stream_t stream) {
-  if (!q || !k || !v || !lse || !dout || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
-  int st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal);
-  if (st) return st;
-  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  const void *ptrs[] = {q, k, v, lse, dout, dk, dv};
+  const void *ptrs[] = {q, k, o, lse, dout};
   for (const void *p : ptrs)
     if (!fa::aligned16(p)) return FA_ERR_ALIGNMENT;
   if (((uintptr_t)workspace & 255u) != 0) return FA_ERR_ALIGNMENT;
   AttnArgs a;
   int dev;
   if ((st = fa::prologue(&dev, a))) return st;
-  a.q = q; a.k = k; a.v = v; a.lse = const_cast<float *>(lse); a.dout = dout;
-  a.dk = dk; a.dv = dv; a.ws = workspace;
+  a.q = q; a.k = k; a.o_in = o; a.lse = const_cast<float *>(lse); a.dout = dout; a.ws = workspace;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.d = d; a.scale = scale;
+  a.stream = (cudaStream_t)stream;
+  return fa::launch_bwd_prep_bf16(a);
+}
+
+FA_EXPORT int fa_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
+                          void *dk, void *dv, void *workspace, int B, int Hq, int Hkv, int Nq,
+                          int Nk, int d, float scale, int causal, fa_stream_t stream) {
+  if (!q || !k || !v || !dout || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  int st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal);
+  if (st) return st;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  const void *ptrs[] = {q, k, v, dout, dk, dv};
+  for (const void *p : ptrs)
+    if (!fa::aligned16(p)) return FA_ERR_ALIGNMENT;
+  if (((uintptr_t)workspace & 255u) != 0) return FA_ERR_ALIGNMENT;
+  AttnArgs a;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.dk = dk; a.dv = dv; a.ws = workspace;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.d = d;
   a.scale = scale; a.causal = causal ? 1 : 0; a.stream = (cudaStream_t)stream;
   return fa::launch_bwd_dkdv_bf16_sm100(a);

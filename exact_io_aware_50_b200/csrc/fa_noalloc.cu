@@ -23,8 +23,8 @@
 #include "common.cuh"
 #include "launch.h"
 
-// 32 MiB: the backward scratch is 4*B*Hq*Nq*(d + 1) bytes (plus padding), so
-// this covers e.g. B*Hq*Nq <= 65,000 query rows at d = 128.
+// 32 MiB: the backward scratch is about 4*B*Hq*(Nq*(d + 2) + d) bytes (plus
+// padding), so this covers e.g. B*Hq*Nq <= 64,000 query rows at d = 128.
 static constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;
 static __device__ __align__(256) unsigned char fa_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -60,7 +60,7 @@ extern "C" __attribute__((visibility("default"))) int fa_bwd_noalloc(
     if (!aligned16(p)) return FA_ERR_ALIGNMENT;
   // Scratch needed for this problem; refuse (before touching the device)
   // anything the fixed array cannot hold.
-  const double need = (double)fa::ws_dq_offset(B, Hq, Nq) + 4.0 * B * Hq * (double)Nq * d;
+  const double need = (double)fa::ws_bytes(B, Hq, Nq, d);
   if (need > (double)kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
   fa::AttnArgs a;
   int dev;

@@ -72,9 +72,11 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
 
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd and fa_bwd_f32
- * need: the per-row vector D = rowsum(dO * O) (B*Hq*Nq float32, rounded up
- * to 256 bytes) followed by a float32 dQ accumulator (B*Hq*Nq*d float32).
- * Returns 0 for invalid sizes.
+ * need (float32 throughout): the per-row vector D = rowsum(dO * O) and the
+ * per-row base-2 log-sum-exp used by the backward, each padded to a multiple
+ * of 64 rows per head; one centring vector per head (B*Hq*d); and a dQ
+ * accumulator (B*Hq*Nq*d), 256-byte aligned.  About 4*B*Hq*(Nq*(d+2) + d)
+ * bytes.  Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
 
@@ -94,18 +96,21 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
  * The three stages fa_bwd runs, exposed so a caller can time or schedule
  * them separately.  Called in this order on one stream with the same
  * workspace they compute exactly what fa_bwd computes (BF16 only):
- *   fa_bwd_prep  -- D = rowsum(dout * o) into the workspace, dQ accumulator
- *                   zeroed;
+ *   fa_bwd_prep  -- per key/value head the centring vector c (the mean of its
+ *                   first 64 key rows, rounded to integers); per query row
+ *                   D = rowsum(dout * o) and the base-2 log-sum-exp shifted
+ *                   by scale * q . c; the dQ accumulator zeroed;
  *   fa_bwd_dkdv  -- the main pass: dk, dv written, dQ accumulated (f32) in
  *                   the workspace;
  *   fa_bwd_dq    -- dq = bf16(scale * accumulator).
  * Same argument rules as fa_bwd.
  */
-int fa_bwd_prep(const void *o, const void *dout, void *workspace, int B, int Hq, int Nq, int d,
+int fa_bwd_prep(const void *q, const void *k, const void *o, const float *lse, const void *dout,
+                void *workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
                 fa_stream_t stream);
-int fa_bwd_dkdv(const void *q, const void *k, const void *v, const float *lse, const void *dout,
-                void *dk, void *dv, void *workspace, int B, int Hq, int Hkv, int Nq, int Nk,
-                int d, float scale, int causal, fa_stream_t stream);
+int fa_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout, void *dk,
+                void *dv, void *workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                float scale, int causal, fa_stream_t stream);
 int fa_bwd_dq(const void *workspace, void *dq, int B, int Hq, int Nq, int d, float scale,
               fa_stream_t stream);
 
@@ -131,8 +136,8 @@ int fa_bwd_f32(const float *q, const float *k, const float *v, const float *o,
  * inside the library (reserved on every GPU that loads it, until exit).
  * The pages have no counterpart; this is an interface convenience.
  * Returns FA_ERR_UNSUPPORTED, without touching the device, when the problem
- * needs more scratch than that (4*B*Hq*Nq*(d+1) bytes plus padding, e.g. more
- * than about 65,000 query rows B*Hq*Nq at d = 128).  The first call on a
+ * needs more scratch than that (about 4*B*Hq*(Nq*(d+2) + d) bytes plus
+ * padding, e.g. more than about 64,000 query rows B*Hq*Nq at d = 128).  The first call on a
  * device looks up the array's address, so make it before any stream capture.
  * Every call uses the same array: calls whose kernels overlap on the GPU
  * (other streams or threads on the same device) race and must be ordered by

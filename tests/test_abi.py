@@ -45,12 +45,16 @@ def test_strerror_covers_codes():
     assert F.fa_strerror(99) == "unknown status"
 
 
+def _ws_expected(B, H, N, d):
+    npad = (N + 63) // 64 * 64
+    head = 2 * B * H * npad * 4 + B * H * d * 4
+    return (head + 255) // 256 * 256 + B * H * N * d * 4
+
+
 def test_workspace_size():
-    B, H, N, d = 4, 16, 4096, 128
-    dbytes = B * H * N * 4
-    assert F.fa_bwd_workspace_size(B, H, N, d) == ((dbytes + 255) // 256) * 256 + B * H * N * d * 4
+    for (B, H, N, d) in ((4, 16, 4096, 128), (1, 1, 3, 64), (2, 3, 1000, 256), (1, 32, 16384, 128)):
+        assert F.fa_bwd_workspace_size(B, H, N, d) == _ws_expected(B, H, N, d)
     assert F.fa_bwd_workspace_size(0, 1, 1, 64) == 0
-    assert F.fa_bwd_workspace_size(1, 1, 3, 64) == 256 + 3 * 64 * 4
 
 
 FAKE = 1 << 20  # 16-byte aligned non-null address; never dereferenced (rejected first)
