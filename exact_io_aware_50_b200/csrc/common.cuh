@@ -21,7 +21,8 @@ namespace fa {
 constexpr long long kWaitLimitNs = 1000000000LL;
 
 enum ErrorBits : unsigned {
-  kErrTimeout = 1u,
+  kErrTimeout = 1u,   // a bounded wait expired
+  kErrConfig = 2u,    // a kernel refused to run (e.g. misaligned shared memory)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -21,11 +21,12 @@
 // Launches on the caller's stream:
 //   prep   1. c per (batch, key/value head) into the workspace;
 //          2. per query row: D_i, L2_i = log2e * L_i - scale * log2e * q_i . c,
-//             padded to 64-row blocks, and the zeroed f32 dQ accumulator;
+//             padded to 128-row blocks, and the zeroed f32 dQ accumulator;
 //   dkdv   one CTA per (batch, key/value head, 128-row key block); K - c and
 //          V stay in shared memory and dK, dV in TMEM for the whole loop over
-//          the query heads of the group and their 64-row query blocks, so dK
-//          and dV need no atomics.  Per step (key rows on the 128 TMEM lanes):
+//          the query heads of the group and their query blocks (128 rows;
+//          64 for d = 256), so dK and dV need no atomics.  Per step (key rows
+//          on the 128 TMEM lanes):
 //              S^T = (K-c) Q_i^T      dP^T = V dO_i^T       (tcgen05, SMEM x SMEM)
 //              P^T = exp2(S^T * scale*log2e - L2_i),  dS^T = P^T * (dP^T - D_i)
 //                                                           (one thread per key row
@@ -33,9 +34,10 @@
 //              dV += P^T dO_i         dK += dS^T Q_i        (tcgen05, A from TMEM)
 //              dQ_i^T = (K-c)^T dS^T                        (tcgen05, SMEM x SMEM)
 //          and a readout warpgroup adds dQ_i^T into the f32 accumulator with
-//          float32 reductions.  Two TMEM score sets let S^T/dP^T of step i+1
-//          run while step i is in its elementwise stage; Q_i, dO_i and the
-//          row vectors L2_i, D_i arrive through a ring of TMA copies;
+//          float32 reductions.  MMA order per step: dV, dK, dQ^T (i), then
+//          S^T (i+1), then -- once dQ^T (i) is in registers -- dP^T (i+1),
+//          which takes dQ^T's TMEM columns.  Q_i, dO_i and the row vectors
+//          L2_i, D_i arrive through a ring of TMA copies;
 //   dq     dQ = bf16(scale * accumulator).
 // For d = 256 the dK and dV accumulators alone fill TMEM, so dkdv runs two
 // passes over the same key blocks: dV (S^T, P^T, dV), then dK and dQ.
@@ -49,25 +51,33 @@
 namespace fa {
 namespace {
 
-// Warp roles: 0-7 elementwise stage (two warpgroups, 32 query columns each),
-// 8-11 dQ readout, 12 TMA producer, 13 MMA issuer.
+// Warp roles: 0-7 elementwise stage (two warpgroups, half of the query
+// columns each, 32 at a time; each also reads out and reduces a quarter of
+// dQ^T), 8-11 dQ readout (the other half of dQ^T), 12 TMA producer, 13 MMA
+// issuer.
 constexpr int kThreads = 448;
 constexpr int kReadoutWarp0 = 8;
 constexpr int kProducerWarp = 12;
 constexpr int kMmaWarp = 13;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kCenterRows = 64;   // key rows averaged into the centring vector c
-constexpr int kRowBlock = 64;     // query rows per step (matches the workspace padding)
 
 enum Mode { kFull = 0, kDV = 1, kDKDQ = 2 };
 
-template <int D_, int MODE_>
+// BM_ query rows per step (MMA N), NSETS_ TMEM score sets, QS_ depth of the
+// Q/dO ring.  An M = 128 tcgen05 MMA takes about as long for N = 64 as for
+// N = 128, but with N = 128 the scores of one step fill the TMEM left next to
+// dK and dV (one set), so MMA and elementwise work cannot overlap.
+template <int D_, int MODE_, int BM_, int NSETS_, int QS_>
 struct BwdCfg {
   static constexpr int D = D_, MODE = MODE_;
   static constexpr int BN = 128;         // key rows per CTA (MMA M)
-  static constexpr int BM = kRowBlock;   // query rows per step (MMA N)
-  static constexpr int NSETS = MODE == kDKDQ ? 1 : 2;   // TMEM score sets
-  static constexpr int QS = MODE == kDKDQ ? 1 : (MODE == kDV ? 2 : (D == 64 ? 4 : 3));
+  static constexpr int BM = BM_;
+  static constexpr int NSETS = NSETS_;
+  static constexpr int QS = QS_;
+  static_assert(BM == 64 || BM == 128, "query block");
+  // dQ^T is written over the dP^T columns (full pass) or into its own columns
+  static constexpr bool DQ_IN_DP = MODE == kFull;
   static constexpr bool HAS_DP = MODE != kDV;
   static constexpr bool HAS_DV = MODE != kDKDQ;
   static constexpr bool HAS_DK = MODE != kDV;
@@ -77,9 +87,9 @@ struct BwdCfg {
   static constexpr int KV_TILE = KV_CHUNK * DCH;
   static constexpr int Q_CHUNK = BM * 128;
   static constexpr int Q_TILE = Q_CHUNK * DCH;
-  static constexpr int DS_TILE = BN * BM * 2;  // dS^T, bf16, one 128-byte chunk wide
-  static constexpr int ROWVEC = BM * 4;         // bytes of one 64-row slice of L2 or D
-  static_assert(BM == 64, "dS^T buffer is one 64-element swizzle chunk wide");
+  static constexpr int DS_CHUNK = BN * 128;    // 64 query columns of dS^T (bf16)
+  static constexpr int DS_TILE = DS_CHUNK * (BM / 64);
+  static constexpr int ROWVEC = BM * 4;         // bytes of one query block of L2 or D
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_TILE;   // must directly follow K (d = 64 dQ MMA)
   static constexpr int OFF_Q = OFF_V + (HAS_DP ? KV_TILE : 0);
@@ -92,20 +102,27 @@ struct BwdCfg {
   // dq_full[2], dq_empty[2], final, drain
   static constexpr int NBAR = 2 + 2 * QS + 8 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  // TMEM columns.
-  //   kFull : dV [0, D), dK [D, 2D), set x at 2D + 128x:
-  //           S^T [0,64) dP^T [64,128); then, for query columns 32w..32w+31
-  //           (warpgroup w), P^T at [32w, 32w+16) and dS^T at [32w+16, 32w+32);
-  //           dQ^T [64,128)
+  // The dynamic shared window starts 1024-byte aligned (checked at run time),
+  // so no alignment slack is reserved.
+  static constexpr int SMEM = OFF_MISC + 16;
+  // TMEM columns (a "set" holds the scores of one step).
+  //   kFull : dV [0, D), dK [D, 2D), set at 2D: S^T [0,128) dP^T [128,256);
+  //           after the elementwise stage, for query columns 32h..32h+31:
+  //           P^T at [32h, 32h+16), dS^T at [32h+16, 32h+32); dQ^T [128,256)
   //   kDV   : dV [0, 256), set x at 256 + 64x: S^T [0,64); then P^T as above
   //   kDKDQ : dK [0, 256), set at 256: S^T [0,64) dP^T [64,128); then dS^T
   //           as above, dQ^T halves [128,192) and [192,256)
   static constexpr int TM_DV = 0;
   static constexpr int TM_DK = MODE == kFull ? D : 0;
   static constexpr int TM_SET0 = MODE == kFull ? 2 * D : D;
-  static constexpr int SET_STRIDE = MODE == kDV ? 64 : 128;
-  static constexpr int TM_DQ = MODE == kFull ? 64 : 128;   // dQ^T offset inside its set
+  static constexpr int SET_STRIDE = MODE == kDV ? BM : 2 * BM;
+  static constexpr int TM_DP = BM;                          // dP^T offset inside a set
+  static constexpr int TM_DQ = MODE == kFull ? BM : 128;    // dQ^T offset inside a set
+  static constexpr int NHALF = D == 256 ? 2 : 1;            // dQ^T pieces of 128 rows of d
+  static constexpr int NCH = NHALF * BM / 32;               // 32-column chunks of dQ^T
+  // the readout warpgroup reads dQ^T chunks 0, 1; the elementwise warpgroups
+  // chunks 2, 3 when a step has four
+  static constexpr int DQ_READERS = (NHALF * BM / 32) == 4 ? 384 : 128;
   static constexpr int TM_ALLOC = 512;
   static_assert(TM_SET0 + NSETS * SET_STRIDE + (MODE == kDKDQ ? 128 : 0) <= TM_ALLOC, "TMEM");
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -134,14 +151,32 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
+// Add 32 columns of dQ^T (one thread = one row d of a 128-row piece of dQ^T,
+// chunk ch of the step's dQ^T columns) into the f32 accumulator.
+template <class C>
+__device__ __forceinline__ void reduce_dq_chunk(const uint32_t (&v)[32], float *acc_row, int ch,
+                                                int d_local, int nvalid) {
+  const int half = (ch * 32) / C::BM;   // which 128 rows of d
+  const int cq = (ch * 32) % C::BM;     // first query column of the chunk
+  if (d_local >= C::D) return;          // d = 64: lanes 64..127 carry no dQ
+  float *a = acc_row + half * 128 + (size_t)cq * C::D;
+#pragma unroll
+  for (int c = 0; c < 32; ++c)
+    if (cq + c < nvalid) atomicAdd(a + (size_t)c * C::D, __uint_as_float(v[c]));
+}
+
 template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                const BwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte aligned base, kept in the shared address space
-  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  // The 128-byte swizzled tiles need a 1024-byte aligned base.
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrConfig);
+    return;
+  }
+  uint8_t *smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
   uint64_t *bars = (uint64_t *)(smem + C::OFF_BAR);
   auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -183,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_SFULL + x), 1);
       mbar_init(bar(B_PFULL + x), 256);
       mbar_init(bar(B_DQFULL + x), 1);
-      mbar_init(bar(B_DQEMPTY + x), 128);
+      mbar_init(bar(B_DQEMPTY + x), C::DQ_READERS);
     }
     mbar_init(bar(B_FINAL), 1);
     mbar_init(bar(B_DRAIN), 1);
@@ -253,9 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t IDESC_SP = idesc_bf16(128, C::BM, 0, 0);  // S^T, dP^T: K-major A and B
     constexpr uint32_t IDESC_KV = idesc_bf16(128, C::D, 0, 1);   // dV, dK: A TMEM, B MN-major
     constexpr uint32_t IDESC_DQ = idesc_bf16(128, C::BM, 1, 1);  // dQ^T: both MN-major
-    auto issue_SdP = [&](int x, int st) {
+    auto issue_S = [&](int x, int st) {
       const uint32_t qa = sbase + C::OFF_Q + st * C::Q_TILE;
-      const uint32_t da = sbase + C::OFF_DO + st * C::Q_TILE;
       const uint32_t set = tmem + C::TM_SET0 + x * C::SET_STRIDE;
 #pragma unroll
       for (int kk = 0; kk < C::D / 16; ++kk) {
@@ -264,20 +298,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_ss(set, sw128_desc(sbase + C::OFF_K + okv, 16, 1024), sw128_desc(qa + oq, 16, 1024),
                IDESC_SP, kk > 0);
       }
-      if (C::HAS_DP) {
+    };
+    auto issue_dP = [&](int x, int st) {
+      if (!C::HAS_DP) return;
+      const uint32_t da = sbase + C::OFF_DO + st * C::Q_TILE;
+      const uint32_t set = tmem + C::TM_SET0 + x * C::SET_STRIDE;
 #pragma unroll
-        for (int kk = 0; kk < C::D / 16; ++kk) {
-          const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
-          const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
-          mma_ss(set + 64, sw128_desc(sbase + C::OFF_V + okv, 16, 1024),
-                 sw128_desc(da + oq, 16, 1024), IDESC_SP, kk > 0);
-        }
+      for (int kk = 0; kk < C::D / 16; ++kk) {
+        const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
+        const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
+        mma_ss(set + C::TM_DP, sw128_desc(sbase + C::OFF_V + okv, 16, 1024),
+               sw128_desc(da + oq, 16, 1024), IDESC_SP, kk > 0);
       }
     };
-    // dV += P^T dO_i and dK += dS^T Q_i (K = 64 query rows, 16 per MMA).
-    // Query rows 16 kk .. 16 kk + 15 of P^T / dS^T live in the columns of the
-    // warpgroup that produced them: P^T at 32 w + [0, 16), dS^T at
-    // 32 w + [16, 32), w = kk / 2.
+    // dV += P^T dO_i and dK += dS^T Q_i (K = BM query rows, 16 per MMA).
+    // Query rows 16 kk .. 16 kk + 15 of P^T / dS^T live in the 32-column block
+    // h = kk / 2 that produced them: P^T at 32 h + [0, 16), dS^T at
+    // 32 h + [16, 32).
     auto issue_dvdk = [&](int x, int st, bool first) {
       const uint32_t qa = sbase + C::OFF_Q + st * C::Q_TILE;
       const uint32_t da = sbase + C::OFF_DO + st * C::Q_TILE;
@@ -295,19 +332,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                  sw128_desc(qa + kk * 2048, C::Q_CHUNK, 1024), IDESC_KV, (!first) || kk > 0);
       }
     };
-    // dQ_i^T = A^T dS^T with K = 128 key rows (16 per MMA) and M = 128 rows of
-    // A^T: [(K-c)^T ; V^T] for d = 64 (the V half is unused), (K-c)^T for
-    // d = 128, and the two 128-row halves of (K-c)^T for d = 256.
+    // dQ_i^T = A^T dS^T with K = 128 key rows (16 per MMA), N = BM query
+    // columns and M = 128 rows of A^T: [(K-c)^T ; V^T] for d = 64 (the V half
+    // is unused), (K-c)^T for d = 128, and the two 128-row halves of (K-c)^T
+    // for d = 256.
     auto issue_dq = [&](int x) {
       const uint32_t set = tmem + C::TM_SET0 + x * C::SET_STRIDE;
       const uint32_t dsb = sbase + C::OFF_DS + x * C::DS_TILE;
 #pragma unroll
-      for (int half = 0; half < (C::D == 256 ? 2 : 1); ++half) {
+      for (int half = 0; half < C::NHALF; ++half) {
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_ss(set + C::TM_DQ + half * 64,
+          mma_ss(set + C::TM_DQ + half * C::BM,
                  sw128_desc(sbase + C::OFF_K + half * 2 * C::KV_CHUNK + kk * 2048, C::KV_CHUNK, 1024),
-                 sw128_desc(dsb + kk * 2048, C::DS_TILE, 1024), IDESC_DQ, kk > 0);
+                 sw128_desc(dsb + kk * 2048, C::DS_CHUNK, 1024), IDESC_DQ, kk > 0);
       }
     };
     // K - c must be in place before the first MMA reads K
@@ -317,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         if (lane == 0) {
-          issue_SdP(0, 0);
+          issue_S(0, 0);
+          issue_dP(0, 0);
           mma_commit(bar(B_SFULL + 0));
         }
         __syncwarp();
@@ -337,14 +376,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
-          issue_SdP(y, st1);
+          issue_S(y, st1);
+          issue_dP(y, st1);
           mma_commit(bar(B_SFULL + y));
         }
         __syncwarp();
       }
       ok = warp_wait_one(bar(B_PFULL + x), set_phase(i), wc);
       if (!ok) break;
-      if (C::HAS_DQ && C::NSETS == 1 && i >= 1) {
+      if (C::HAS_DQ && C::NSETS == 1 && !C::DQ_IN_DP && i >= 1) {
         ok = warp_wait_one(bar(B_DQEMPTY + x), set_phase(i - 1), wc);
         if (!ok) break;
       }
@@ -359,12 +399,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (C::NSETS == 1 && i + 1 < nsteps) {
+        // S^T(i+1) only overwrites P^T/dS^T, which dV/dK(i) (issued earlier)
+        // consume in order; dP^T(i+1) overwrites dQ^T(i) when they share
+        // columns, so it waits for the readout of dQ^T(i).
         const int st1 = (i + 1) % C::QS;
         ok = warp_wait_one(bar(B_QFULL + st1), ((i + 1) / C::QS) & 1, wc);
         if (!ok) break;
         tc_fence_after();
+        if (lane == 0) issue_S(x, st1);
+        __syncwarp();
+        if (C::HAS_DQ && C::DQ_IN_DP) {
+          ok = warp_wait_one(bar(B_DQEMPTY + x), set_phase(i), wc);
+          if (!ok) break;
+          tc_fence_after();
+        }
         if (lane == 0) {
-          issue_SdP(x, st1);
+          issue_dP(x, st1);
           mma_commit(bar(B_SFULL + x));
         }
         __syncwarp();
@@ -416,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(bar(B_KC));
     }
-    const int c0 = wg * 32;
+    constexpr int NCB = C::BM / 64;   // 32-column blocks per warpgroup and step
     for (int i = 0; i < nsteps && ok; ++i) {
       const int x = set_of(i), st = i % C::QS;
       ok = warp_wait_all(bar(B_QFULL + st), (i / C::QS) & 1, wc);
@@ -424,62 +474,85 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t set = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE;
-      uint32_t sv[32], dv[32];
-      tmem_ld32(set + c0, sv);
-      if (C::HAS_DP) tmem_ld32(set + 64 + c0, dv);
-      tmem_wait_ld();
-      const float4 *l4 = reinterpret_cast<const float4 *>(s_l2 + st * C::BM + c0);
-      const float4 *d4 = reinterpret_cast<const float4 *>(s_dd + st * C::BM + c0);
-      const int q0 = step_qblk(i) * C::BM + c0;
-      // causal: key kv is hidden from query q when kv > q; key rows past Nk
-      // (zero-filled) are masked so they add nothing anywhere.  Query rows
-      // past Nq have L2 = +inf, so their P is 0.
-      const int first_vis = !kv_live ? 32 : (p.causal ? kv - q0 : 0);
-      const bool unmasked = __all_sync(0xffffffffu, first_vis <= 0);
-      uint32_t pk[16], dk[16];
-      auto body = [&](auto masked_tag) {
-        constexpr bool MASKED = decltype(masked_tag)::value;
+#pragma unroll 1
+      for (int hh = 0; hh < NCB; ++hh) {
+        const int cb = wg * NCB + hh;   // 32-column block of the step
+        const int c0 = cb * 32;
+        uint32_t sv[32], dv[32];
+        tmem_ld32(set + c0, sv);
+        if (C::HAS_DP) tmem_ld32(set + C::TM_DP + c0, dv);
+        tmem_wait_ld();
+        const float4 *l4 = reinterpret_cast<const float4 *>(s_l2 + st * C::BM + c0);
+        const float4 *d4 = reinterpret_cast<const float4 *>(s_dd + st * C::BM + c0);
+        const int q0 = step_qblk(i) * C::BM + c0;
+        // causal: key kv is hidden from query q when kv > q; key rows past
+        // Nk (zero-filled) are masked so they add nothing anywhere.  Query
+        // rows past Nq have L2 = +inf, so their P is 0.
+        const int first_vis = !kv_live ? 32 : (p.causal ? kv - q0 : 0);
+        const bool unmasked = __all_sync(0xffffffffu, first_vis <= 0);
+        uint32_t pk[16], dk[16];
+        auto body = [&](auto masked_tag) {
+          constexpr bool MASKED = decltype(masked_tag)::value;
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 lq = l4[e4];
-          const float4 dq4 = C::HAS_DP ? d4[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
-          const float dvv[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
-          float pr[4], ds[4];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 lq = l4[e4];
+            const float4 dq4 = C::HAS_DP ? d4[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
+            const float dvv[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
+            float pr[4], ds[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = 4 * e4 + u;
-            float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[u]));
-            if (MASKED) pv = (c >= first_vis) ? pv : 0.f;
-            pr[u] = pv;
-            ds[u] = C::HAS_DP ? pv * (__uint_as_float(dv[c]) - dvv[u]) : 0.f;
+            for (int u = 0; u < 4; ++u) {
+              const int c = 4 * e4 + u;
+              float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[u]));
+              if (MASKED) pv = (c >= first_vis) ? pv : 0.f;
+              pr[u] = pv;
+              ds[u] = C::HAS_DP ? pv * (__uint_as_float(dv[c]) - dvv[u]) : 0.f;
+            }
+            pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
+            pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
+            dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+            dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
           }
-          pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
-          pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
-          dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
-          dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
-        }
-      };
-      if (unmasked) body(std::false_type{});
-      else body(std::true_type{});
-      // bf16 P^T and dS^T go into this warpgroup's own (already read) S^T
-      // columns, so the other warpgroup's unread columns are never touched
-      if (C::HAS_DV) tmem_st16(set + c0, pk);
-      if (C::HAS_DK) tmem_st16(set + c0 + 16, dk);
-      if (C::HAS_DQ) {
-        // dS^T row r -> shared memory (B operand of the dQ^T MMA, 128-byte
-        // swizzled rows: 16-byte chunk c of row r sits at chunk c ^ (r % 8));
-        // this warpgroup owns chunks 4 wg .. 4 wg + 3
-        uint8_t *dsrow = smem + C::OFF_DS + x * C::DS_TILE + r * 128;
+        };
+        if (unmasked) body(std::false_type{});
+        else body(std::true_type{});
+        // bf16 P^T and dS^T go into the 32 S^T columns just read, so columns
+        // another thread group has not read yet are never touched
+        if (C::HAS_DV) tmem_st16(set + c0, pk);
+        if (C::HAS_DK) tmem_st16(set + c0 + 16, dk);
+        if (C::HAS_DQ) {
+          // dS^T row r -> shared memory (B operand of the dQ^T MMA: 64-column
+          // chunks of 128-byte swizzled rows; 16-byte unit u of row r sits
+          // at unit u ^ (r % 8))
+          uint8_t *dsrow = smem + C::OFF_DS + x * C::DS_TILE + (c0 >> 6) * C::DS_CHUNK + r * 128;
+          const int u0 = (c0 & 63) >> 3;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4 *>(dsrow + (((4 * wg + c) ^ (r & 7)) << 4)) =
-              make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
-        fence_proxy_async_smem();
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4 *>(dsrow + (((u0 + c) ^ (r & 7)) << 4)) =
+                make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+        }
       }
+      if (C::HAS_DQ) fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PFULL + x));
+      if (C::HAS_DQ && C::NCH == 4) {
+        // Share of the dQ^T readout: chunk 2 + wg (the readout warpgroup takes
+        // chunks 0 and 1), so every column is in registers before dQ^T's TMEM
+        // columns are released, with room to spare.
+        ok = warp_wait_all(bar(B_DQFULL + x), set_phase(i), wc);
+        if (!ok) break;
+        tc_fence_after();
+        const int ch = 2 + wg;
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ + ch * 32, v);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_DQEMPTY + x));
+        const int qb0 = step_qblk(i) * C::BM;
+        float *acc = p.dq_acc + (((size_t)(b * p.Hq + step_head(i))) * p.Nq + qb0) * C::D + r;
+        reduce_dq_chunk<C>(v, acc, ch, r, min(C::BM, p.Nq - qb0));
+      }
     }
     // ------------------------------------------------------ epilogue
     // warpgroup 0 writes dV, warpgroup 1 writes dK (one key row per thread)
@@ -515,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ dQ readout
     const int t = threadIdx.x - 32 * kReadoutWarp0;  // TMEM lane = column d of dQ (per half)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    static_assert(C::NCH == 2 || C::NCH == 4, "dQ^T readout split");
     for (int i = 0; i < nsteps; ++i) {
       const int x = set_of(i);
       if (!warp_wait_all(bar(B_DQFULL + x), set_phase(i), wc)) break;
@@ -522,25 +596,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = step_head(i), q0 = step_qblk(i) * C::BM;
       const int nvalid = min(C::BM, p.Nq - q0);
       float *acc = p.dq_acc + (((size_t)(b * p.Hq + h)) * p.Nq + q0) * C::D + t;
-      constexpr int NH = C::D == 256 ? 2 : 1;
-#pragma unroll 1
-      for (int half = 0; half < NH; ++half) {
-        uint32_t v[64];
-        const uint32_t src = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ + half * 64;
-        tmem_ld32(src, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(src + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_wait_ld();
-        if (half == NH - 1) {
-          tc_fence_before();
-          mbar_arrive(bar(B_DQEMPTY + x));
-        }
-        if (t < C::D) {
-          float *a = acc + half * 128;
-#pragma unroll
-          for (int c = 0; c < C::BM; ++c)
-            if (c < nvalid) atomicAdd(a + (size_t)c * C::D, __uint_as_float(v[c]));
-        }
-      }
+      const uint32_t src = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ;
+      // chunks 0 and 1 (the elementwise warpgroups take chunks 2 and 3)
+      uint32_t v0[32], v1[32];
+      tmem_ld32(src, v0);
+      tmem_ld32(src + 32, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_DQEMPTY + x));
+      reduce_dq_chunk<C>(v0, acc, 0, t, nvalid);
+      reduce_dq_chunk<C>(v1, acc, 1, t, nvalid);
     }
   }
 
@@ -727,13 +792,23 @@ int launch_bwd_prep_bf16(const AttnArgs &a) {
   }
 }
 
+#ifndef FA_BWD_BM
+#define FA_BWD_BM 64
+#endif
+#ifndef FA_BWD_NSETS
+#define FA_BWD_NSETS 2
+#endif
+#ifndef FA_BWD_QS
+#define FA_BWD_QS 4
+#endif
+#define FA_BWD_FULL_CFG FA_BWD_BM, FA_BWD_NSETS, FA_BWD_QS
 int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {
-    case 64: return run_dkdv<BwdCfg<64, kFull>>(a);
-    case 128: return run_dkdv<BwdCfg<128, kFull>>(a);
+    case 64: return run_dkdv<BwdCfg<64, kFull, FA_BWD_FULL_CFG>>(a);
+    case 128: return run_dkdv<BwdCfg<128, kFull, FA_BWD_FULL_CFG>>(a);
     case 256: {
-      int st = run_dkdv<BwdCfg<256, kDV>>(a);
-      return st ? st : run_dkdv<BwdCfg<256, kDKDQ>>(a);
+      int st = run_dkdv<BwdCfg<256, kDV, 64, 2, 2>>(a);
+      return st ? st : run_dkdv<BwdCfg<256, kDKDQ, 64, 1, 1>>(a);
     }
     default: return 2;
   }

@@ -283,7 +283,8 @@ FA_EXPORT int fa_device_status(fa_stream_t stream) {
     return FA_ERR_CUDA;
   if (host && cudaMemcpy(err, &zero, sizeof(unsigned), cudaMemcpyHostToDevice) != cudaSuccess)
     return FA_ERR_CUDA;
-  return (host & fa::kErrTimeout) ? FA_ERR_TIMEOUT : FA_OK;
+  if (host & fa::kErrTimeout) return FA_ERR_TIMEOUT;
+  return host ? FA_ERR_CUDA : FA_OK;
 }
 
 FA_EXPORT int fa_wait_selftest(long long timeout_ns, fa_stream_t stream) {

@@ -27,9 +27,9 @@ struct AttnArgs {
 //                      base 2, shifted for the centred K; rows past Nq +inf
 //   c   [B*Hq][d]      per key/value head centring vector (first B*Hkv*d used)
 //   dQ  [B*Hq][Nq][d]  dQ accumulator, 256-byte aligned
-// Npad = Nq rounded up to 64, so every 64-row slice of D and L2 is a
-// 256-byte aligned block a bulk copy can fetch.
-inline size_t ws_npad(int Nq) { return (size_t)((Nq + 63) / 64) * 64; }
+// Npad = Nq rounded up to 128, so every 64- or 128-row query block of D and
+// L2 is a 256-byte aligned block a bulk copy can fetch.
+inline size_t ws_npad(int Nq) { return (size_t)((Nq + 127) / 128) * 128; }
 inline size_t ws_l2_offset(int B, int Hq, int Nq) { return (size_t)B * Hq * ws_npad(Nq) * 4; }
 inline size_t ws_c_offset(int B, int Hq, int Nq) { return 2 * ws_l2_offset(B, Hq, Nq); }
 inline size_t ws_dq_offset(int B, int Hq, int Nq, int d) {

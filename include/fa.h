@@ -153,7 +153,8 @@ int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
  * library's device error word on the current device.  Returns FA_OK, or
  * FA_ERR_TIMEOUT when a kernel's bounded wait expired since the last call
  * (that kernel then returned early and its outputs are undefined), or
- * FA_ERR_CUDA when the synchronisation itself failed.
+ * FA_ERR_CUDA when the synchronisation itself failed or a kernel refused to
+ * run (its shared memory was not 1024-byte aligned).
  */
 int fa_device_status(fa_stream_t stream);
 

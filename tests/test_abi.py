@@ -46,7 +46,7 @@ def test_strerror_covers_codes():
 
 
 def _ws_expected(B, H, N, d):
-    npad = (N + 63) // 64 * 64
+    npad = (N + 127) // 128 * 128
     head = 2 * B * H * npad * 4 + B * H * d * 4
     return (head + 255) // 256 * 256 + B * H * N * d * 4
 
