@@ -290,6 +290,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
+// Descriptor of the same layout moved forward by `bytes` (a multiple of 16,
+// staying below 256 KiB of shared memory, so the 14-bit field cannot carry).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and f32 accumulator.
 // a_mn / b_mn select MN-major operands (0 = K-major).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
@@ -312,6 +318,27 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x evaluated on the FMA pipe (the MUFU unit that runs ex2 is the
+// softmax's bottleneck, so part of the exponentials go here instead).
+// Range reduction: x = j + f with j the nearest integer -- adding 1.5 * 2^23
+// leaves j in the low mantissa bits of t -- and f in [-1/2, 1/2].  2^f comes
+// from a cubic 1 + f (c1 + f (c2 + f c3)) fitted for minimum relative error
+// on [-1/2, 1/2] with the constant term held at 1, so 2^x is exact at every
+// integer x -- in particular at the row maximum, where x = 0 (maximum
+// relative error 1.02e-4, below bf16 resolution) -- and 2^j is applied by
+// adding j to the exponent field.  Valid for x <= 127; inputs below -126
+// (including -inf) return a value below 2^-125 instead of 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float j = t - 12582912.0f;
+  const float f = x - j;
+  float p = fmaf(0.055008817464113235f, f, 0.24221080541610718f);
+  p = fmaf(p, f, 0.6932829022407532f);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {

@@ -288,27 +288,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t IDESC_SP = idesc_bf16(128, C::BM, 0, 0);  // S^T, dP^T: K-major A and B
     constexpr uint32_t IDESC_KV = idesc_bf16(128, C::D, 0, 1);   // dV, dK: A TMEM, B MN-major
     constexpr uint32_t IDESC_DQ = idesc_bf16(128, C::BM, 1, 1);  // dQ^T: both MN-major
+    // Descriptors are built once; each MMA offsets a base descriptor.
+    const uint64_t dK_km = sw128_desc(sbase + C::OFF_K, 16, 1024);        // K-c, K-major
+    const uint64_t dV_km = sw128_desc(sbase + C::OFF_V, 16, 1024);        // V, K-major
+    const uint64_t dK_mn = sw128_desc(sbase + C::OFF_K, C::KV_CHUNK, 1024);  // (K-c)^T, MN-major
+    const uint64_t dQ_km = sw128_desc(sbase + C::OFF_Q, 16, 1024);
+    const uint64_t dQ_mn = sw128_desc(sbase + C::OFF_Q, C::Q_CHUNK, 1024);
+    const uint64_t dO_km = sw128_desc(sbase + C::OFF_DO, 16, 1024);
+    const uint64_t dO_mn = sw128_desc(sbase + C::OFF_DO, C::Q_CHUNK, 1024);
+    const uint64_t dS_mn = sw128_desc(sbase + C::OFF_DS, C::DS_CHUNK, 1024);
     auto issue_S = [&](int x, int st) {
-      const uint32_t qa = sbase + C::OFF_Q + st * C::Q_TILE;
+      const uint64_t qa = desc_add(dQ_km, st * C::Q_TILE);
       const uint32_t set = tmem + C::TM_SET0 + x * C::SET_STRIDE;
 #pragma unroll
       for (int kk = 0; kk < C::D / 16; ++kk) {
         const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
         const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
-        mma_ss(set, sw128_desc(sbase + C::OFF_K + okv, 16, 1024), sw128_desc(qa + oq, 16, 1024),
-               IDESC_SP, kk > 0);
+        mma_ss(set, desc_add(dK_km, okv), desc_add(qa, oq), IDESC_SP, kk > 0);
       }
     };
     auto issue_dP = [&](int x, int st) {
       if (!C::HAS_DP) return;
-      const uint32_t da = sbase + C::OFF_DO + st * C::Q_TILE;
+      const uint64_t da = desc_add(dO_km, st * C::Q_TILE);
       const uint32_t set = tmem + C::TM_SET0 + x * C::SET_STRIDE;
 #pragma unroll
       for (int kk = 0; kk < C::D / 16; ++kk) {
         const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
         const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
-        mma_ss(set + C::TM_DP, sw128_desc(sbase + C::OFF_V + okv, 16, 1024),
-               sw128_desc(da + oq, 16, 1024), IDESC_SP, kk > 0);
+        mma_ss(set + C::TM_DP, desc_add(dV_km, okv), desc_add(da, oq), IDESC_SP, kk > 0);
       }
     };
     // dV += P^T dO_i and dK += dS^T Q_i (K = BM query rows, 16 per MMA).
@@ -316,20 +323,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // h = kk / 2 that produced them: P^T at 32 h + [0, 16), dS^T at
     // 32 h + [16, 32).
     auto issue_dvdk = [&](int x, int st, bool first) {
-      const uint32_t qa = sbase + C::OFF_Q + st * C::Q_TILE;
-      const uint32_t da = sbase + C::OFF_DO + st * C::Q_TILE;
+      const uint64_t qa = desc_add(dQ_mn, st * C::Q_TILE);
+      const uint64_t da = desc_add(dO_mn, st * C::Q_TILE);
       const uint32_t set = tmem + C::TM_SET0 + x * C::SET_STRIDE;
       if (C::HAS_DV) {
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk)
-          mma_ts(tmem + C::TM_DV, set + (kk >> 1) * 32 + (kk & 1) * 8,
-                 sw128_desc(da + kk * 2048, C::Q_CHUNK, 1024), IDESC_KV, (!first) || kk > 0);
+          mma_ts(tmem + C::TM_DV, set + (kk >> 1) * 32 + (kk & 1) * 8, desc_add(da, kk * 2048),
+                 IDESC_KV, (!first) || kk > 0);
       }
       if (C::HAS_DK) {
 #pragma unroll
         for (int kk = 0; kk < C::BM / 16; ++kk)
           mma_ts(tmem + C::TM_DK, set + (kk >> 1) * 32 + 16 + (kk & 1) * 8,
-                 sw128_desc(qa + kk * 2048, C::Q_CHUNK, 1024), IDESC_KV, (!first) || kk > 0);
+                 desc_add(qa, kk * 2048), IDESC_KV, (!first) || kk > 0);
       }
     };
     // dQ_i^T = A^T dS^T with K = 128 key rows (16 per MMA), N = BM query
@@ -338,14 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // for d = 256.
     auto issue_dq = [&](int x) {
       const uint32_t set = tmem + C::TM_SET0 + x * C::SET_STRIDE;
-      const uint32_t dsb = sbase + C::OFF_DS + x * C::DS_TILE;
+      const uint64_t dsb = desc_add(dS_mn, x * C::DS_TILE);
 #pragma unroll
       for (int half = 0; half < C::NHALF; ++half) {
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
           mma_ss(set + C::TM_DQ + half * C::BM,
-                 sw128_desc(sbase + C::OFF_K + half * 2 * C::KV_CHUNK + kk * 2048, C::KV_CHUNK, 1024),
-                 sw128_desc(dsb + kk * 2048, C::DS_CHUNK, 1024), IDESC_DQ, kk > 0);
+                 desc_add(dK_mn, half * 2 * C::KV_CHUNK + kk * 2048), desc_add(dsb, kk * 2048),
+                 IDESC_DQ, kk > 0);
       }
     };
     // K - c must be in place before the first MMA reads K

@@ -39,6 +39,13 @@ constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+#ifndef FA_FWD_POLY_EXP
+#define FA_FWD_POLY_EXP 0
+#endif
+// When on, one column in four of P takes its exponential from exp2_poly (FMA
+// pipe) instead of MUFU.  Off by default: on B200 it measured 3-5% slower
+// than MUFU alone, so the exponential unit is not what bounds this kernel.
+constexpr bool kPolyExp = FA_FWD_POLY_EXP != 0;
 
 template <int D_, int NT_, int BN_, int STAGES_>
 struct FwdCfg {
@@ -186,24 +193,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t IDESC_S = idesc_bf16(BM, C::BN, 0, 0);
     constexpr uint32_t IDESC_PV = idesc_bf16(BM, C::D, 0, 1);
+    // Descriptors are built once; each MMA offsets a base descriptor.
+    const uint64_t dq0 = sw128_desc(sbase + C::OFF_Q, 16, 1024);
+    const uint64_t dk0 = sw128_desc(sbase + C::OFF_K, 16, 1024);
+    const uint64_t dv0 = sw128_desc(sbase + C::OFF_V, C::KV_CHUNK, 1024);
     auto issue_S = [&](int t, int s) {
-      const uint32_t qa = sbase + C::OFF_Q + t * C::Q_TILE;
-      const uint32_t kb = sbase + C::OFF_K + s * C::KV_TILE;
+      const uint64_t qa = desc_add(dq0, t * C::Q_TILE);
+      const uint64_t kb = desc_add(dk0, s * C::KV_TILE);
 #pragma unroll
       for (int kk = 0; kk < C::D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
         const uint32_t offk = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
-        mma_ss(tmem + C::TM_S + t * C::BN, sw128_desc(qa + off, 16, 1024),
-               sw128_desc(kb + offk, 16, 1024), IDESC_S, kk > 0);
+        mma_ss(tmem + C::TM_S + t * C::BN, desc_add(qa, off), desc_add(kb, offk), IDESC_S,
+               kk > 0);
       }
     };
     auto issue_PV = [&](int t, int s, bool first) {
-      const uint32_t vb = sbase + C::OFF_V + s * C::KV_TILE;
+      const uint64_t vb = desc_add(dv0, s * C::KV_TILE);
       const uint32_t pcol = tmem + C::TM_S + t * C::BN + C::BN / 2;
 #pragma unroll
       for (int kk = 0; kk < C::BN / 16; ++kk) {
-        mma_ts(tmem + C::TM_O + t * C::D, pcol + kk * 8,
-               sw128_desc(vb + kk * 16 * 128, C::KV_CHUNK, 1024), IDESC_PV, (!first) || kk > 0);
+        mma_ts(tmem + C::TM_O + t * C::D, pcol + kk * 8, desc_add(vb, kk * 16 * 128),
+               IDESC_PV, (!first) || kk > 0);
       }
     };
     bool ok = warp_wait_one(bar(B_QFULL), 0, wc);
@@ -285,9 +296,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < C::BN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
       }
-      float mx = s[0];
+      // row max: eight independent partial maxima, then a small tree
+      float mp[8];
 #pragma unroll
-      for (int c = 1; c < C::BN; ++c) mx = fmaxf(mx, s[c]);
+      for (int u = 0; u < 8; ++u) mp[u] = s[u];
+#pragma unroll
+      for (int c = 8; c < C::BN; c += 8)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mp[u] = fmaxf(mp[u], s[c + u]);
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float m_new = fmaxf(m_run, mx * p.scale_log2);
       bool rescale = false;
       float alpha = 1.f;
@@ -299,19 +317,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float rowsum = 0.f;
+      // p = 2^(s * scale * log2e - m): one column in four on the FMA pipe
+      // (exp2_poly), the rest on MUFU; row sum in four independent partials
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < C::BN / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = fast_exp2(fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_use));
-          const float p1 = fast_exp2(fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_use));
-          rowsum += p0 + p1;
+          const float x0 = fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_use);
+          const float x1 = fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_use);
+          const float p0 = fast_exp2(x0);
+          const float p1 = (kPolyExp && (e & 1)) ? exp2_poly(x1) : fast_exp2(x1);
+          rs[e & 3] += p0 + p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tP + c * 16, pk);
       }
+      const float rowsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
       l_run = l_run * alpha + rowsum;
       if (rescale) {
 #pragma unroll 1
