@@ -110,6 +110,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
+# ------------------------------------------------- cross-rank aggregation
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of a list of floats over all ranks (identity alone).
+    Every rank must call it at the same point."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_tflops(world, flops_per_rank_step, ms_per_step):
+    """All ranks' FLOPs over the slowest rank's time, in TFLOP/s."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ ours
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -232,13 +249,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = a0.elapsed_time(a1) / e2e_steps
 
-    if dist is not None:
-        t = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
     ms_per_step = total_ms / args.steps
-    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
-    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, step_flops, ms_per_step)
+    e2e_value = whole_job_tflops(world, step_flops, e2e_ms)
 
     burst, sustained, hbm, src = measured_peaks()
     # dominant kernel by measured share of the step
