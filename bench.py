@@ -318,12 +318,19 @@ def load_traffic(workload, kernel):
 
 
 def source_sha():
+    """Hash of the kernel sources with comments and blank lines removed, so a
+    comment edit does not invalidate recorded counters but a code edit does."""
     import hashlib
+    import re
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "exact_io_aware_50_b200", "csrc")
     for f in sorted(os.listdir(cs)):
-        with open(os.path.join(cs, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(cs, f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+        h.update(f.encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 
