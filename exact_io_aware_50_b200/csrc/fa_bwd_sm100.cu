@@ -192,11 +192,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
 
-  // Work unit: key blocks with the most query blocks first (causal), then
-  // (batch, key/value head).
+  // Work unit: head by head (batch, key/value head), and inside a head the
+  // key blocks with the most query blocks first (causal).  A wave then reads
+  // the Q, dO and dQ-accumulator tiles of a few heads only, which stay in L2.
   const int unit = blockIdx.x;
-  const int jblk = unit / p.BHkv;
-  const int bhkv = unit % p.BHkv;
+  const int jblk = unit % p.nkb;
+  const int bhkv = unit / p.nkb;
   const int b = bhkv / p.Hkv, hkv = bhkv % p.Hkv;
   const int g = p.Hq / p.Hkv;
   const int kv0 = jblk * C::BN;
@@ -622,6 +623,459 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// dkdv for d <= 128 with 128-row query blocks.
+//
+// An M = 128 tcgen05 MMA costs about as much for N = 64 as for N = 128, so
+// S^T, dP^T and dQ^T are computed for 128 query columns at a time.  TMEM then
+// holds dV, dK and one set of scores:
+//     d = 128: dV [0,128) dK [128,256) A [256,384) B [384,512)
+//     d =  64: dV [0, 64) dK [ 64,128) A [128,256) B [256,384)
+// A receives S^T(i), which the elementwise stage overwrites in place with
+// bf16 P^T and dS^T; B receives dP^T(i) and then dQ^T(i).  The elementwise
+// stage runs in two phases so the tensor cores are not left idle while it
+// works:
+//     phase 1 (needs S^T):  P^T = exp2(S^T * scale*log2e - L2)  -> dV(i) may start
+//     phase 2 (needs dP^T): dS^T = P^T * (dP^T - D)            -> dK(i), dQ^T(i)
+// MMA issue order per step:  dV(i)  dK(i)  S^T(i+1)  dQ^T(i)  dP^T(i+1).
+// S^T(i+1) only replaces what dV(i) and dK(i), issued before it, read;
+// dP^T(i+1) waits until the readout warps hold dQ^T(i) in registers.  Phase 1
+// of step i+1 then overlaps dQ^T(i), its readout and dP^T(i+1), and phase 2
+// overlaps dV(i+1).  P^T is kept in registers between the phases in bf16, the
+// precision the dV MMA also uses.
+//
+// Warps: 0-7 elementwise (two warpgroups, 64 query columns each; warpgroup 0
+// writes dV and warpgroup 1 dK at the end), 8-15 dQ^T readout (two warps per
+// TMEM lane quarter, two 32-column chunks each, float32 reductions into the
+// accumulator), 16 TMA producer, 17 MMA issuer (both in lane 0).
+template <int D_, int QS_>
+struct BwdWideCfg {
+  static constexpr int D = D_, QS = QS_;
+  static constexpr int BN = 128, BM = 128;
+  static constexpr int DCH = D / 64;
+  static constexpr int KV_CHUNK = BN * 128;
+  static constexpr int KV_TILE = KV_CHUNK * DCH;
+  static constexpr int Q_CHUNK = BM * 128;
+  static constexpr int Q_TILE = Q_CHUNK * DCH;
+  static constexpr int DS_CHUNK = BN * 128;        // 64 query columns of dS^T (bf16)
+  static constexpr int DS_TILE = DS_CHUNK * 2;
+  static constexpr int ROWVEC = BM * 4;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_TILE;    // must directly follow K (d = 64 dQ MMA)
+  static constexpr int OFF_Q = OFF_V + KV_TILE;
+  static constexpr int OFF_DO = OFF_Q + QS * Q_TILE;
+  static constexpr int OFF_DS = OFF_DO + QS * Q_TILE;
+  static constexpr int OFF_L2 = OFF_DS + DS_TILE;
+  static constexpr int OFF_DD = OFF_L2 + QS * ROWVEC;
+  static constexpr int OFF_BAR = OFF_DD + QS * ROWVEC;
+  // kv, kc, q_full[QS], q_empty[QS], s_full, dp_full, p_full, ds_full,
+  // dq_full, dq_empty, final, drain
+  static constexpr int NBAR = 2 + 2 * QS + 8;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16;
+  static constexpr int TM_DV = 0, TM_DK = D, TM_A = 2 * D, TM_B = 2 * D + 128;
+  static constexpr int TM_ALLOC = 512;
+  static constexpr int THREADS = 18 * 32;
+  static constexpr int READOUT_WARP0 = 8, PRODUCER_WARP = 16, MMA_WARP = 17;
+  static_assert(TM_B + 128 <= TM_ALLOC, "TMEM");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(D == 64 || D == 128, "wide path is for d = 64 and 128");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    bwd_wide_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte swizzled tiles need a 1024-byte aligned base.
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrConfig);
+    return;
+  }
+  uint8_t *smem = smem_raw;
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t *bars = (uint64_t *)(smem + C::OFF_BAR);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int B_KV = 0, B_KC = 1, B_QFULL = 2, B_QEMPTY = 2 + C::QS, B_SFULL = 2 + 2 * C::QS,
+            B_DPFULL = B_SFULL + 1, B_PFULL = B_SFULL + 2, B_DSFULL = B_SFULL + 3,
+            B_DQFULL = B_SFULL + 4, B_DQEMPTY = B_SFULL + 5, B_FINAL = B_SFULL + 6,
+            B_DRAIN = B_SFULL + 7;
+  uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
+  volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
+  const float *s_l2 = (const float *)(smem + C::OFF_L2);
+  const float *s_dd = (const float *)(smem + C::OFF_DD);
+
+  const int warp = warp_id_uniform();
+  const int lane = threadIdx.x & 31;
+
+  // Work unit: head by head (batch, key/value head), and inside a head the
+  // key blocks with the most query blocks first (causal).
+  const int unit = blockIdx.x;
+  const int jblk = unit % p.nkb;
+  const int bhkv = unit / p.nkb;
+  const int b = bhkv / p.Hkv, hkv = bhkv % p.Hkv;
+  const int g = p.Hq / p.Hkv;
+  const int kv0 = jblk * C::BN;
+  const int i0 = p.causal ? kv0 / C::BM : 0;  // first query block that sees this key block
+  const int nq_eff = p.nqb - i0;
+  const int nsteps = nq_eff > 0 ? g * nq_eff : 0;
+  auto step_head = [&](int s) { return hkv * g + s / nq_eff; };
+  auto step_qblk = [&](int s) { return i0 + s % nq_eff; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_KV), 1);
+    mbar_init(bar(B_KC), 256);
+    for (int s = 0; s < C::QS; ++s) {
+      mbar_init(bar(B_QFULL + s), 1);
+      mbar_init(bar(B_QEMPTY + s), 1);
+    }
+    mbar_init(bar(B_SFULL), 1);
+    mbar_init(bar(B_DPFULL), 1);
+    mbar_init(bar(B_PFULL), 256);
+    mbar_init(bar(B_DSFULL), 256);
+    mbar_init(bar(B_DQFULL), 1);
+    mbar_init(bar(B_DQEMPTY), 256);
+    mbar_init(bar(B_FINAL), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::TM_ALLOC);
+    tmem_relinquish();
+  }
+  if (warp == C::PRODUCER_WARP && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmDO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  WaitCtx wc{p.err, abort_flag, kWaitLimitNs};
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int last_phase[C::QS];
+      for (int s = 0; s < C::QS; ++s) last_phase[s] = -1;
+      bool ok = true;
+      mbar_arrive_expect_tx(bar(B_KV), 2 * C::KV_TILE);
+      for (int c = 0; c < C::DCH; ++c) {
+        tma_load_3d(sbase + C::OFF_K + c * C::KV_CHUNK, &tmK, bar(B_KV), c * 64, kv0, bhkv);
+        tma_load_3d(sbase + C::OFF_V + c * C::KV_CHUNK, &tmV, bar(B_KV), c * 64, kv0, bhkv);
+      }
+      for (int i = 0; i < nsteps && ok; ++i) {
+        const int st = i % C::QS;
+        const uint32_t ph = (i / C::QS) & 1;
+        ok = bounded_wait(bar(B_QEMPTY + st), ph ^ 1, wc);
+        if (!ok) break;
+        const int h = step_head(i), qb = step_qblk(i);
+        const int bh = b * p.Hq + h;
+        const size_t vrow = (size_t)bh * p.npad + (size_t)qb * C::BM;
+        const uint32_t fb = bar(B_QFULL + st);
+        mbar_arrive_expect_tx(fb, 2 * C::Q_TILE + 2 * C::ROWVEC);
+        for (int c = 0; c < C::DCH; ++c) {
+          tma_load_3d(sbase + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, fb, c * 64,
+                      qb * C::BM, bh);
+          tma_load_3d(sbase + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmDO, fb, c * 64,
+                      qb * C::BM, bh);
+        }
+        bulk_load(sbase + C::OFF_L2 + st * C::ROWVEC, p.l2 + vrow, C::ROWVEC, fb);
+        bulk_load(sbase + C::OFF_DD + st * C::ROWVEC, p.dsum + vrow, C::ROWVEC, fb);
+        last_phase[st] = ph;
+      }
+      if (!ok) {
+        (void)drain_wait(bar(B_KV), 0, p.err, kWaitLimitNs);
+        for (int s = 0; s < C::QS; ++s)
+          if (last_phase[s] >= 0) (void)drain_wait(bar(B_QFULL + s), last_phase[s], p.err, kWaitLimitNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t IDESC_SP = idesc_bf16(128, C::BM, 0, 0);  // S^T, dP^T
+    constexpr uint32_t IDESC_KV = idesc_bf16(128, C::D, 0, 1);   // dV, dK: A TMEM, B MN-major
+    constexpr uint32_t IDESC_DQ = idesc_bf16(128, C::BM, 1, 1);  // dQ^T: both MN-major
+    const uint64_t dK_km = sw128_desc(sbase + C::OFF_K, 16, 1024);
+    const uint64_t dV_km = sw128_desc(sbase + C::OFF_V, 16, 1024);
+    const uint64_t dK_mn = sw128_desc(sbase + C::OFF_K, C::KV_CHUNK, 1024);
+    const uint64_t dQ_km = sw128_desc(sbase + C::OFF_Q, 16, 1024);
+    const uint64_t dQ_mn = sw128_desc(sbase + C::OFF_Q, C::Q_CHUNK, 1024);
+    const uint64_t dO_km = sw128_desc(sbase + C::OFF_DO, 16, 1024);
+    const uint64_t dO_mn = sw128_desc(sbase + C::OFF_DO, C::Q_CHUNK, 1024);
+    const uint64_t dS_mn = sw128_desc(sbase + C::OFF_DS, C::DS_CHUNK, 1024);
+    // S^T = (K-c) Q^T (A region), dP^T = V dO^T (B region); K = d, 16 per MMA
+    auto issue_SP = [&](uint64_t a0, uint64_t b0, int st, uint32_t dst) {
+      const uint64_t bt = desc_add(b0, st * C::Q_TILE);
+#pragma unroll
+      for (int kk = 0; kk < C::D / 16; ++kk) {
+        const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
+        const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
+        mma_ss(dst, desc_add(a0, okv), desc_add(bt, oq), IDESC_SP, kk > 0);
+      }
+    };
+    // dV += P^T dO_i, dK += dS^T Q_i: K = 128 query rows, 16 per MMA; query
+    // rows 16 kk .. 16 kk + 15 sit in the 32-column block kk / 2 of A: P^T at
+    // 32 (kk / 2) + 8 (kk % 2), dS^T 16 columns further.
+    auto issue_grad = [&](uint64_t b0, int st, uint32_t acc, int col, bool first) {
+      const uint64_t bt = desc_add(b0, st * C::Q_TILE);
+#pragma unroll
+      for (int kk = 0; kk < C::BM / 16; ++kk)
+        mma_ts(tmem + acc, tmem + C::TM_A + (kk >> 1) * 32 + (kk & 1) * 8 + col,
+               desc_add(bt, kk * 2048), IDESC_KV, (!first) || kk > 0);
+    };
+    // dQ^T = A^T dS^T, K = 128 key rows (16 per MMA), M = 128 rows of A^T:
+    // (K-c)^T for d = 128, [(K-c)^T ; V^T] for d = 64 (the V half unused).
+    auto issue_dq = [&]() {
+#pragma unroll
+      for (int kk = 0; kk < C::BN / 16; ++kk)
+        mma_ss(tmem + C::TM_B, desc_add(dK_mn, kk * 2048), desc_add(dS_mn, kk * 2048), IDESC_DQ,
+               kk > 0);
+    };
+    if (lane == 0) {
+      bool ok = bounded_wait(bar(B_KC), 0, wc);   // K - c in place
+      if (ok && nsteps > 0) {
+        ok = bounded_wait(bar(B_QFULL + 0), 0, wc);
+        if (ok) {
+          tc_fence_after();
+          issue_SP(dK_km, dQ_km, 0, tmem + C::TM_A);
+          mma_commit(bar(B_SFULL));
+          issue_SP(dV_km, dO_km, 0, tmem + C::TM_B);
+          mma_commit(bar(B_DPFULL));
+        }
+      }
+      for (int i = 0; i < nsteps && ok; ++i) {
+        const int st = i % C::QS;
+        const uint32_t par = i & 1;
+        ok = bounded_wait(bar(B_PFULL), par, wc);
+        if (!ok) break;
+        tc_fence_after();
+        issue_grad(dO_mn, st, C::TM_DV, 0, i == 0);
+        ok = bounded_wait(bar(B_DSFULL), par, wc);
+        if (!ok) break;
+        tc_fence_after();
+        issue_grad(dQ_mn, st, C::TM_DK, 16, i == 0);
+        mma_commit(bar(B_QEMPTY + st));
+        const int st1 = (i + 1) % C::QS;
+        if (i + 1 < nsteps) {
+          ok = bounded_wait(bar(B_QFULL + st1), ((i + 1) / C::QS) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_SP(dK_km, dQ_km, st1, tmem + C::TM_A);
+          mma_commit(bar(B_SFULL));
+        }
+        issue_dq();
+        mma_commit(bar(B_DQFULL));
+        if (i + 1 < nsteps) {
+          ok = bounded_wait(bar(B_DQEMPTY), par, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_SP(dV_km, dO_km, st1, tmem + C::TM_B);
+          mma_commit(bar(B_DPFULL));
+        }
+      }
+      if (ok) {
+        mma_commit(bar(B_FINAL));
+      } else {
+        mma_commit(bar(B_DRAIN));
+        (void)drain_wait(bar(B_DRAIN), 0, p.err, kWaitLimitNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp < C::READOUT_WARP0) {
+    // ------------------------------------------------ elementwise stage
+    const int wg = warp >> 2;                      // query columns [64 wg, 64 wg + 64)
+    const int r = threadIdx.x & 127;               // key row within the block = TMEM lane
+    const int kv = kv0 + r;
+    const bool kv_live = kv < p.Nk;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    bool ok = warp_wait_all(bar(B_KV), 0, wc);
+    if (ok) {
+      // K row r -> K - c in place (same swizzled layout; rows past Nk were
+      // zero-filled and stay zero).  Warpgroup wg takes chunks wg, wg + 2, ...
+      const float *cv = p.cvec + (size_t)bhkv * C::D;
+#pragma unroll 1
+      for (int ch = wg; ch < C::DCH; ch += 2) {
+        uint8_t *row = smem + C::OFF_K + ch * C::KV_CHUNK + r * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int col = ch * 64 + ((u ^ (r & 7)) << 3);
+          const float4 c_lo = *reinterpret_cast<const float4 *>(cv + col);
+          const float4 c_hi = *reinterpret_cast<const float4 *>(cv + col + 4);
+          const float cc[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
+          uint4 v = *reinterpret_cast<const uint4 *>(row + (u << 4));
+          uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+            const float2 f = __bfloat1622float2(h2);
+            w[e] = kv_live ? pack_bf16x2(f.x - cc[2 * e], f.y - cc[2 * e + 1]) : 0u;
+          }
+          *reinterpret_cast<uint4 *>(row + (u << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_KC));
+    }
+    const uint32_t tA = tmem + lane_off + C::TM_A;
+    const uint32_t tB = tmem + lane_off + C::TM_B;
+    for (int i = 0; i < nsteps && ok; ++i) {
+      const int st = i % C::QS;
+      const uint32_t par = i & 1;
+      const int q0 = step_qblk(i) * C::BM;
+      ok = warp_wait_all(bar(B_QFULL + st), (i / C::QS) & 1, wc);
+      if (ok) ok = warp_wait_all(bar(B_SFULL), par, wc);
+      if (!ok) break;
+      tc_fence_after();
+      // ---- phase 1: P^T for query columns [64 wg, 64 wg + 64), 16 at a time
+      uint32_t pkeep[4][8];
+#pragma unroll
+      for (int sb = 0; sb < 4; ++sb) {
+        const int c0 = 64 * wg + 16 * sb;
+        uint32_t sv[16];
+        tmem_ld16(tA + c0, sv);
+        tmem_wait_ld();
+        const float4 *l4 = reinterpret_cast<const float4 *>(s_l2 + st * C::BM + c0);
+        // causal: key kv is hidden from query q when kv > q; key rows past
+        // Nk (zero-filled) are masked so they add nothing anywhere.  Query
+        // rows past Nq have L2 = +inf, so their P is 0.
+        const int first_vis = !kv_live ? 16 : (p.causal ? kv - (q0 + c0) : 0);
+        float pr[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const float4 lq = l4[e4];
+          const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = 4 * e4 + u;
+            const float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[u]));
+            pr[c] = (c >= first_vis) ? pv : 0.f;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pkeep[sb][e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+        // P^T of query columns 32h + 16(sb%2) + [0,16) -> A columns 32h + 8(sb%2) + [0,8),
+        // all of which this thread has already read
+        tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 8 * (sb & 1), pkeep[sb]);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL));
+      // ---- phase 2: dS^T = P^T (dP^T - D)
+      ok = warp_wait_all(bar(B_DPFULL), par, wc);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int sb = 0; sb < 4; ++sb) {
+        const int c0 = 64 * wg + 16 * sb;
+        uint32_t dv[16];
+        tmem_ld16(tB + c0, dv);
+        tmem_wait_ld();
+        const float4 *d4 = reinterpret_cast<const float4 *>(s_dd + st * C::BM + c0);
+        uint32_t dk[8];
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const float4 dq4 = d4[e4];
+          const float dd[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
+          float ds[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = 4 * e4 + u;
+            const uint32_t pp = pkeep[sb][c >> 1];
+            const float pv = __uint_as_float((c & 1) ? (pp & 0xffff0000u) : (pp << 16));
+            ds[u] = pv * (__uint_as_float(dv[c]) - dd[u]);
+          }
+          dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+          dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
+        }
+        tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 16 + 8 * (sb & 1), dk);
+        // dS^T row r -> shared memory (B operand of the dQ^T MMA: 64-column
+        // chunks of 128-byte swizzled rows; 16-byte unit u of row r sits at
+        // unit u ^ (r % 8))
+        uint8_t *dsrow = smem + C::OFF_DS + (c0 >> 6) * C::DS_CHUNK + r * 128;
+        const int u0 = (c0 & 63) >> 3;
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          *reinterpret_cast<uint4 *>(dsrow + (((u0 + c) ^ (r & 7)) << 4)) =
+              make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_DSFULL));
+    }
+    // ------------------------------------------------------ epilogue
+    // warpgroup 0 writes dV, warpgroup 1 writes dK (one key row per thread)
+    if (ok) ok = warp_wait_all(bar(B_FINAL), 0, wc);
+    if (ok && nsteps > 0) {
+      tc_fence_after();
+      const size_t rowoff = ((size_t)bhkv * p.Nk + (kv_live ? kv : 0)) * C::D;
+      const uint32_t src = tmem + lane_off + (wg ? C::TM_DK : C::TM_DV);
+      __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + rowoff;
+      const float mul = wg ? p.scale : 1.f;
+#pragma unroll 1
+      for (int c = 0; c < C::D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(src + c * 32, v);
+        tmem_wait_ld();
+        uint32_t pkd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pkd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+        if (kv_live) {
+          uint4 *o = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+        }
+      }
+    } else if (ok && nsteps == 0 && kv_live) {
+      // no query row sees this key block: its gradients are zero
+      __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + ((size_t)bhkv * p.Nk + kv) * C::D;
+      for (int e = 0; e < C::D / 8; ++e) reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0, 0, 0, 0);
+    }
+  } else if (warp < C::PRODUCER_WARP) {
+    // ------------------------------------------------ dQ^T readout
+    const int quad = warp & 3;
+    const int t = quad * 32 + lane;                  // TMEM lane = row d of dQ^T
+    const int ch0 = ((warp - C::READOUT_WARP0) >> 2) * 2;   // chunks ch0, ch0 + 1
+    const uint32_t src = tmem + ((uint32_t)(quad * 32) << 16) + C::TM_B + ch0 * 32;
+    for (int i = 0; i < nsteps; ++i) {
+      if (!warp_wait_all(bar(B_DQFULL), i & 1, wc)) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      const bool live_rows = quad * 32 < C::D;    // d = 64: lanes 64..127 carry no dQ
+      if (live_rows) {
+        tmem_ld32(src, v0);
+        tmem_ld32(src + 32, v1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_DQEMPTY));
+      if (!live_rows) continue;
+      const int h = step_head(i), q0 = step_qblk(i) * C::BM;
+      const int nvalid = min(C::BM, p.Nq - q0);
+      float *acc = p.dq_acc + (((size_t)(b * p.Hq + h)) * p.Nq + q0 + ch0 * 32) * C::D + t;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (ch0 * 32 + c < nvalid) atomicAdd(acc + (size_t)c * C::D, __uint_as_float(v0[c]));
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (ch0 * 32 + 32 + c < nvalid) atomicAdd(acc + (size_t)(32 + c) * C::D, __uint_as_float(v1[c]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_ALLOC);
+  }
+}
+
 // c[b, hkv, :] = mean of the head's first min(Nk, 64) key rows, rounded to
 // integers (f32).  One CTA per (batch, key/value head), one thread per column.
 template <int D>
@@ -743,7 +1197,7 @@ int run_prep(const AttnArgs &a) {
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }
 
-template <class C>
+template <class C, bool WIDE>
 int run_dkdv(const AttnArgs &a) {
   const WsPtrs w = ws_ptrs(a);
   CUtensorMap mq, mk, mv, mdo;
@@ -768,13 +1222,21 @@ int run_dkdv(const AttnArgs &a) {
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
   p.err = a.err;
-  auto kern = bwd_kernel<C>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
-      cudaSuccess)
-    return 5;
   const long long units = (long long)p.nkb * p.BHkv;
   if (units > 2147483647LL) return 2;
-  kern<<<(unsigned)units, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
+  if constexpr (WIDE) {
+    auto kern = bwd_wide_kernel<C>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+      return 5;
+    kern<<<(unsigned)units, C::THREADS, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
+  } else {
+    auto kern = bwd_kernel<C>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+      return 5;
+    kern<<<(unsigned)units, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
+  }
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }
 
@@ -807,13 +1269,21 @@ int launch_bwd_prep_bf16(const AttnArgs &a) {
 #define FA_BWD_QS 4
 #endif
 #define FA_BWD_FULL_CFG FA_BWD_BM, FA_BWD_NSETS, FA_BWD_QS
+#ifndef FA_BWD_WIDE
+#define FA_BWD_WIDE 1
+#endif
 int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {
-    case 64: return run_dkdv<BwdCfg<64, kFull, FA_BWD_FULL_CFG>>(a);
-    case 128: return run_dkdv<BwdCfg<128, kFull, FA_BWD_FULL_CFG>>(a);
+#if FA_BWD_WIDE
+    case 64: return run_dkdv<BwdWideCfg<64, 4>, true>(a);
+    case 128: return run_dkdv<BwdWideCfg<128, 2>, true>(a);
+#else
+    case 64: return run_dkdv<BwdCfg<64, kFull, FA_BWD_FULL_CFG>, false>(a);
+    case 128: return run_dkdv<BwdCfg<128, kFull, FA_BWD_FULL_CFG>, false>(a);
+#endif
     case 256: {
-      int st = run_dkdv<BwdCfg<256, kDV, 64, 2, 2>>(a);
-      return st ? st : run_dkdv<BwdCfg<256, kDKDQ, 64, 1, 1>>(a);
+      int st = run_dkdv<BwdCfg<256, kDV, 64, 2, 2>, false>(a);
+      return st ? st : run_dkdv<BwdCfg<256, kDKDQ, 64, 1, 1>, false>(a);
     }
     default: return 2;
   }

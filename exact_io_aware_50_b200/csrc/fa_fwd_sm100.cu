@@ -106,10 +106,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
 
-  // Work unit: heavy query blocks first (causal), then (batch, head).
+  // Work unit.  Causal: the heaviest query blocks of every head first, so the
+  // last wave holds the shortest units.  Otherwise all units cost the same and
+  // they run head by head, so the K and V tiles a wave reads are those of a
+  // few heads and stay in L2.
   const int unit = blockIdx.x;
-  const int qblk = p.nqb - 1 - unit / p.BH;
-  const int bh = unit % p.BH;
+  const int qblk = p.causal ? p.nqb - 1 - unit / p.BH : unit % p.nqb;
+  const int bh = p.causal ? unit % p.BH : unit / p.nqb;
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int bh_kv = b * p.Hkv + h / (p.Hq / p.Hkv);
   const int q_start = qblk * C::NT * BM;
