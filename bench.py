@@ -286,7 +286,9 @@ def run_ours(args, rank, world, local_rank):
                      "unit": "TFLOP/s", "frac": round(achieved / burst, 4), "traffic": traffic},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": 4 * args.steps,
+        # per step: forward; prep = centring + preprocess; dkdv (two passes
+        # at d = 256); dq conversion
+        "gpu_launches": (1 + 2 + (2 if w.d == 256 else 1) + 1) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
