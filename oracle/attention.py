@@ -26,6 +26,17 @@ What it computes (the plain definition, materialised, in float64):
 * Grouped-query attention (GQA, named in the wiki's FlashAttention-2 history):
   query head h reads key/value head floor(h / g), g = Hq / Hkv; dK and dV of a
   key/value head sum over the g query heads of its group.
+* Causal alignment when Nq < Nk (inference: the Nq queries are the last Nq
+  positions of a sequence whose Nk keys are all cached) -- the pages only use
+  Nq = Nk.  Reading adopted: bottom-right alignment, key j is masked for
+  query i when j > i + (Nk - Nq); it equals the top-left mask when Nq = Nk.
+  Selected with ``causal_offset = Nk - Nq``; the default 0 is top-left.
+* Split-KV forward and the merge of partial results -- the key range of a
+  row is cut into pieces, each piece gives (O_s, L_s) over its own keys, and
+  the pieces are combined with the same rescaling identity that the online
+  softmax of blog section 2.2 uses to combine two blocks' statistics:
+      L = log sum_s exp(L_s),   O = sum_s exp(L_s - L) O_s.
+  A piece that sees no key of a row has L_s = -inf and contributes nothing.
 * Block-wise forms -- the online-softmax step of blog section 2.2 (normalise at
   every block, "v1") and the deferred-normalisation loop of blog section 4.1
   and the CSDN tutorial section 3 ("v2": keep O unnormalised, rescale by
@@ -54,6 +65,8 @@ __all__ = [
     "backward_kv_rows",
     "blockwise_forward_v1",
     "blockwise_forward_v2",
+    "merge_partials",
+    "splitkv_forward",
 ]
 
 
@@ -68,33 +81,34 @@ def _kv_head(h: int, hq: int, hkv: int) -> int:
     return h // (hq // hkv)
 
 
-def _causal_mask(nq: int, nk: int) -> np.ndarray:
-    """True where key j is hidden from query i (j > i, top-left alignment)."""
+def _causal_mask(nq: int, nk: int, offset: int = 0) -> np.ndarray:
+    """True where key j is hidden from query i: j > i + offset (offset 0:
+    top-left alignment; offset Nk - Nq: bottom-right)."""
     i = np.arange(nq)[:, None]
     j = np.arange(nk)[None, :]
-    return j > i
+    return j > i + offset
 
 
-def scores(q2, k2, scale, causal):
+def scores(q2, k2, scale, causal, causal_offset=0):
     """Masked scaled scores S = scale * q k^T for one head; masked entries -inf.
 
     Standard attention, blog section 1; causal mask per blog section 5."""
     s = scale * (_f64(q2) @ _f64(k2).T)
     if causal:
-        s = np.where(_causal_mask(s.shape[0], s.shape[1]), -np.inf, s)
+        s = np.where(_causal_mask(s.shape[0], s.shape[1], causal_offset), -np.inf, s)
     return s
 
 
-def probs(q2, k2, scale, causal):
+def probs(q2, k2, scale, causal, causal_offset=0):
     """P = softmax(S) row-wise, max-subtracted (blog section 2.2)."""
-    s = scores(q2, k2, scale, causal)
+    s = scores(q2, k2, scale, causal, causal_offset)
     m = np.max(s, axis=1, keepdims=True)
     e = np.exp(s - m)
     return e / np.sum(e, axis=1, keepdims=True)
 
 
-def _head_forward(q2, k2, v2, scale, causal):
-    s = scores(q2, k2, scale, causal)
+def _head_forward(q2, k2, v2, scale, causal, causal_offset=0):
+    s = scores(q2, k2, scale, causal, causal_offset)
     m = np.max(s, axis=1, keepdims=True)
     e = np.exp(s - m)
     l = np.sum(e, axis=1, keepdims=True)
@@ -104,7 +118,7 @@ def _head_forward(q2, k2, v2, scale, causal):
     return o, lse, p
 
 
-def forward(q, k, v, scale, causal):
+def forward(q, k, v, scale, causal, causal_offset=0):
     """O = softmax(scale * Q K^T [+ causal mask]) V and L = logsumexp per row.
 
     q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d].  Returns (o [B,Hq,Nq,d],
@@ -117,7 +131,8 @@ def forward(q, k, v, scale, causal):
     for b in range(B):
         for h in range(Hq):
             kh = _kv_head(h, Hq, Hkv)
-            o[b, h], lse[b, h], _ = _head_forward(q[b, h], k[b, kh], v[b, kh], scale, causal)
+            o[b, h], lse[b, h], _ = _head_forward(q[b, h], k[b, kh], v[b, kh], scale, causal,
+                                                  causal_offset)
     return o, lse
 
 
@@ -154,17 +169,18 @@ def backward(q, k, v, do, scale, causal):
 # so an N x N matrix never has to exist at once.
 # ---------------------------------------------------------------------------
 
-def _row_chunk_scores(q2, k2, scale, causal, rows):
+def _row_chunk_scores(q2, k2, scale, causal, rows, causal_offset=0):
     s = scale * (_f64(q2)[rows] @ _f64(k2).T)
     if causal:
-        s = np.where(np.arange(k2.shape[0])[None, :] > np.asarray(rows)[:, None], -np.inf, s)
+        s = np.where(np.arange(k2.shape[0])[None, :] > np.asarray(rows)[:, None] + causal_offset,
+                     -np.inf, s)
     return s
 
 
-def forward_rows(q2, k2, v2, scale, causal, rows):
+def forward_rows(q2, k2, v2, scale, causal, rows, causal_offset=0):
     """O and L for the given query rows of one head (q2 [Nq,d], k2/v2 [Nk,d])."""
     rows = np.asarray(rows)
-    s = _row_chunk_scores(q2, k2, scale, causal, rows)
+    s = _row_chunk_scores(q2, k2, scale, causal, rows, causal_offset)
     m = np.max(s, axis=1, keepdims=True)
     e = np.exp(s - m)
     l = np.sum(e, axis=1, keepdims=True)
@@ -280,3 +296,61 @@ def blockwise_forward_v2(q2, k2, v2, scale, causal, block):
         l = alpha * l + np.sum(e, axis=1, keepdims=True)
         m = m_new
     return o_t / l, (m + np.log(l))[:, 0]
+
+
+# ---------------------------------------------------------------------------
+# Split-KV forward: partial results over key ranges, merged by their LSE.
+# ---------------------------------------------------------------------------
+
+def merge_partials(o_parts, lse_parts):
+    """Combine per-piece results of the same rows.
+
+    o_parts [S, ..., d] holds each piece's normalised output over its own keys,
+    lse_parts [S, ...] its log-sum-exp (-inf where the piece sees no key of the
+    row).  Returns (o, lse) with lse = log sum_s exp(lse_s) and
+    o = sum_s exp(lse_s - lse) o_s (the block-combination identity of blog
+    section 2.2, applied to normalised pieces)."""
+    o_parts, lse_parts = _f64(o_parts), _f64(lse_parts)
+    m = np.max(lse_parts, axis=0)
+    safe = np.where(np.isneginf(m), 0.0, m)
+    w = np.where(np.isneginf(lse_parts), 0.0, np.exp(lse_parts - safe))
+    tot = np.sum(w, axis=0)
+    lse = safe + np.log(tot)
+    o = np.sum(w[..., None] * o_parts, axis=0) / tot[..., None]
+    return o, lse
+
+
+def splitkv_forward(q, k, v, scale, causal, bounds, causal_offset=0):
+    """Forward by pieces of the key range, then merge_partials.
+
+    bounds: increasing key indices [0 = b_0, b_1, ..., b_S = Nk]; piece s covers
+    keys [b_s, b_{s+1}).  Returns (o, lse, o_parts, lse_parts).  Each piece is
+    the plain definition restricted to its keys (rows with no visible key in a
+    piece get lse = -inf and o = 0)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    S = len(bounds) - 1
+    o_parts = np.zeros((S, B, Hq, Nq, v.shape[3]))
+    lse_parts = np.full((S, B, Hq, Nq), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            kh = _kv_head(h, Hq, Hkv)
+            s_full = scores(q[b, h], k[b, kh], scale, causal, causal_offset)
+            for p_ in range(S):
+                j0, j1 = bounds[p_], bounds[p_ + 1]
+                sp = s_full[:, j0:j1]
+                if sp.shape[1] == 0:
+                    continue
+                m = np.max(sp, axis=1, keepdims=True)
+                live = ~np.isneginf(m[:, 0])
+                safe = np.where(np.isneginf(m), 0.0, m)
+                e = np.where(np.isneginf(sp), 0.0, np.exp(sp - safe))
+                l = np.sum(e, axis=1, keepdims=True)
+                with np.errstate(invalid="ignore", divide="ignore"):
+                    op = np.where(live[:, None], (e @ v[b, kh, j0:j1]) / np.where(l > 0, l, 1.0), 0.0)
+                    lp = np.where(live, (safe + np.log(np.where(l > 0, l, 1.0)))[:, 0], -np.inf)
+                o_parts[p_, b, h] = op
+                lse_parts[p_, b, h] = lp
+    o, lse = merge_partials(o_parts, lse_parts)
+    return o, lse, o_parts, lse_parts

@@ -23,7 +23,9 @@ RNG = np.random.default_rng(1234)
 def real_impl():
     return types.SimpleNamespace(forward=OA.forward, backward=OA.backward, probs=OA.probs,
                                  forward_rows=OA.forward_rows, backward_rows=OA.backward_rows,
-                                 backward_kv_rows=OA.backward_kv_rows, lse_rows=OA.lse_rows)
+                                 backward_kv_rows=OA.backward_kv_rows, lse_rows=OA.lse_rows,
+                                 merge_partials=lambda o, l: OA.merge_partials(o, l),
+                                 splitkv_forward=lambda *a, **kw: OA.splitkv_forward(*a, **kw))
 
 
 def rnd(*shape, scale=1.0):
@@ -242,9 +244,63 @@ def pin_row_forms(impl):
             np.testing.assert_allclose(dvr, dv[0, kh, kv_rows], atol=1e-12)
 
 
+def pin_bottom_right(impl):
+    """Bottom-right causal alignment (key j hidden from query i when
+    j > i + Nk - Nq): a single query sees every key (= non-causal); the Nq
+    queries equal the last Nq rows of the square top-left problem whatever
+    precedes them; offset 0 is the top-left mask."""
+    nk, d = 11, 4
+    k, v = rnd(1, 1, nk, d), rnd(1, 1, nk, d)
+    q1 = rnd(1, 1, 1, d)
+    o_c, l_c = impl.forward(q1, k, v, 0.6, True, nk - 1)
+    o_n, l_n = impl.forward(q1, k, v, 0.6, False)
+    np.testing.assert_allclose(o_c, o_n, atol=1e-14)
+    np.testing.assert_allclose(l_c, l_n, atol=1e-14)
+    for nq in (3, 7, nk):
+        q = rnd(1, 1, nq, d)
+        qpad = np.concatenate([rnd(1, 1, nk - nq, d), q], axis=2)
+        o_sq, l_sq = impl.forward(qpad, k, v, 0.6, True)
+        o_br, l_br = impl.forward(q, k, v, 0.6, True, nk - nq)
+        np.testing.assert_allclose(o_br, o_sq[:, :, nk - nq:], atol=1e-13)
+        np.testing.assert_allclose(l_br, l_sq[:, :, nk - nq:], atol=1e-13)
+        p = impl.probs(q[0, 0], k[0, 0], 0.6, True, nk - nq)
+        i, j = np.meshgrid(np.arange(nq), np.arange(nk), indexing="ij")
+        assert np.all(p[j > i + nk - nq] == 0) and np.all(p[j <= i + nk - nq] > 0)
+
+
+def pin_merge_partials(impl):
+    """Split-KV: pieces over any cut of the key range (empty pieces, one-key
+    pieces, pieces a causal row cannot see) merge to the one-shot result; the
+    two-piece merge equals its closed form; piece order does not matter."""
+    nq, nk, d = 6, 19, 4
+    q, k, v = rnd(2, 2, nq, d), rnd(2, 1, nk, d), rnd(2, 1, nk, d)
+    for causal, off in ((False, 0), (True, nk - nq)):
+        o, l = impl.forward(q, k, v, 0.5, causal, off)
+        for bounds in ([0, nk], [0, 1, nk], [0, 5, 5, 12, 18, nk], [0, 15, 17, nk]):
+            o_s, l_s, op, lp = impl.splitkv_forward(q, k, v, 0.5, causal, bounds, off)
+            np.testing.assert_allclose(o_s, o, atol=1e-13)
+            np.testing.assert_allclose(l_s, l, atol=1e-13)
+            perm = np.arange(len(bounds) - 1)[::-1]
+            o_p, l_p = impl.merge_partials(op[perm], lp[perm])
+            np.testing.assert_allclose(o_p, o, atol=1e-13)
+            np.testing.assert_allclose(l_p, l, atol=1e-13)
+    o1, o2 = rnd(3, d), rnd(3, d)
+    l1, l2 = rnd(3), rnd(3)
+    om, lm = impl.merge_partials(np.stack([o1, o2]), np.stack([l1, l2]))
+    w1, w2 = np.exp(l1), np.exp(l2)
+    np.testing.assert_allclose(om, (w1[:, None] * o1 + w2[:, None] * o2) / (w1 + w2)[:, None],
+                               atol=1e-14)
+    np.testing.assert_allclose(lm, np.log(w1 + w2), atol=1e-14)
+    oe, le = impl.merge_partials(np.stack([o1, np.zeros_like(o1)]),
+                                 np.stack([l1, np.full(3, -np.inf)]))
+    np.testing.assert_allclose(oe, o1, atol=1e-15)
+    np.testing.assert_allclose(le, l1, atol=1e-15)
+
+
 PINS = [pin_probs_rows, pin_constant_v, pin_causal_row0, pin_zero_q, pin_single_key,
         pin_shift_invariance, pin_kplus8_bf16, pin_gradient_identities, pin_permutation,
-        pin_hand_example, pin_finite_differences, pin_torch_sdpa, pin_row_forms]
+        pin_hand_example, pin_finite_differences, pin_torch_sdpa, pin_row_forms,
+        pin_bottom_right, pin_merge_partials]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -303,12 +359,14 @@ def _mutant(name):
     impl = real_impl()
     patches = {}
     if name == "mask_includes_diagonal":
-        patches["_causal_mask"] = lambda nq, nk: np.arange(nk)[None, :] >= np.arange(nq)[:, None]
+        patches["_causal_mask"] = lambda nq, nk, offset=0: (np.arange(nk)[None, :] >=
+                                                            np.arange(nq)[:, None] + offset)
     elif name == "mask_off_by_one_late":
-        patches["_causal_mask"] = lambda nq, nk: np.arange(nk)[None, :] > np.arange(nq)[:, None] + 1
+        patches["_causal_mask"] = lambda nq, nk, offset=0: (np.arange(nk)[None, :] >
+                                                            np.arange(nq)[:, None] + offset + 1)
     elif name == "scale_dropped":
         orig = OA.scores
-        patches["scores"] = lambda q2, k2, scale, causal: orig(q2, k2, 1.0, causal)
+        patches["scores"] = lambda q2, k2, scale, causal, off=0: orig(q2, k2, 1.0, causal, off)
     elif name == "lse_log2":
         f = impl.forward
 
@@ -330,6 +388,16 @@ def _mutant(name):
             dq, dk, dv, D = b(q, k, v, do, scale, causal)
             return dq, dk, dv[:, :, ::-1].copy(), D
         impl.backward = bwd
+    elif name == "causal_offset_ignored":
+        patches["_causal_mask"] = lambda nq, nk, offset=0: (np.arange(nk)[None, :] >
+                                                            np.arange(nq)[:, None])
+    elif name == "merge_unweighted":
+        def merge(o_parts, lse_parts):
+            o_parts, lse_parts = np.asarray(o_parts), np.asarray(lse_parts)
+            m = np.max(lse_parts, axis=0)
+            return o_parts.mean(axis=0), m + np.log(np.sum(np.exp(lse_parts - m), axis=0))
+        patches["merge_partials"] = merge
+        impl.merge_partials = merge
     elif name == "gqa_mod_mapping":
         patches["_kv_head"] = lambda h, hq, hkv: h % hkv
     elif name == "D_without_O":
@@ -356,8 +424,8 @@ def _mutant(name):
         impl.backward = bwd
     elif name == "no_max_subtraction_overflow":
         # softmax without the max shift overflows for large scores -> NaN
-        def pr(q2, k2, scale, causal):
-            s = OA.scores(q2, k2, scale, causal) * 1e3
+        def pr(q2, k2, scale, causal, off=0):
+            s = OA.scores(q2, k2, scale, causal, off) * 1e3
             e = np.exp(s)
             return e / e.sum(axis=1, keepdims=True)
         impl.probs = pr
@@ -368,7 +436,7 @@ def _mutant(name):
 
 MUTANTS = ["mask_includes_diagonal", "mask_off_by_one_late", "scale_dropped", "lse_log2",
            "dk_no_scale", "dv_untransposed", "gqa_mod_mapping", "D_without_O",
-           "no_max_subtraction_overflow"]
+           "no_max_subtraction_overflow", "causal_offset_ignored", "merge_unweighted"]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
