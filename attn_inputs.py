@@ -30,10 +30,11 @@ class Workload:
     q_mul: float = 1.0           # Q pre-multiplied in float32 before the cast
     k_add: float = 0.0           # constant added to every K element before the cast
     backward: bool = True
+    n_q: int = 0                 # query rows when fewer than N (inference shapes); 0 -> N
 
     @property
     def Nq(self) -> int:
-        return self.N
+        return self.n_q or self.N
 
     @property
     def Nk(self) -> int:
@@ -69,8 +70,12 @@ TWO_BATCH_BF16 = Workload("two_batch_bf16_n1024_d64", 2, 1, 1, 1024, 64, False, 
 CAUSAL_TRAIN = Workload("causal_b4_h16_n4096_d128", 4, 16, 16, 4096, 128, True, "bf16", 3)
 LONG_GQA = Workload("long_gqa_b1_hq32_hkv8_n16384_d128_q2x", 1, 32, 8, 16384, 128, True, "bf16", 4, q_mul=2.0)
 SWEEP = _c5()
+# Inference shape (forward only, split-KV path): batch 1, 8 heads, 512 new
+# query rows against a 16384-key cache, causal bottom-right aligned.
+INFER_PREFILL = Workload("inference_b1_h8_nq512_nk16384_d128", 1, 8, 8, 16384, 128, True, "bf16", 6,
+                         backward=False, n_q=512)
 
-ALL = [SINGLE_HEAD_F32, TWO_BATCH_F32, TWO_BATCH_BF16, CAUSAL_TRAIN, LONG_GQA] + SWEEP
+ALL = [SINGLE_HEAD_F32, TWO_BATCH_F32, TWO_BATCH_BF16, CAUSAL_TRAIN, LONG_GQA] + SWEEP + [INFER_PREFILL]
 BY_NAME = {w.name: w for w in ALL}
 
 
@@ -84,7 +89,7 @@ def make(w: Workload, *, B=None, Hq=None, Hkv=None, N=None, Nq=None, Nk=None, d=
     Hq = w.Hq if Hq is None else Hq
     Hkv = w.Hkv if Hkv is None else Hkv
     N = w.N if N is None else N
-    Nq = N if Nq is None else Nq
+    Nq = (w.n_q or N) if Nq is None else Nq
     Nk = N if Nk is None else Nk
     d = w.d if d is None else d
     seed = w.seed if seed is None else seed

@@ -16,6 +16,11 @@ the max over ranks and the value is the sum of all ranks' FLOPs over it.
 
 ``--impl reference`` times the float64 CPU oracle (the only reference there
 is) on a bounded sample of the same workload and prints the same JSON line.
+
+``--workload inference_b1_h8_nq512_nk16384_d128`` (or any forward-only
+workload with fewer query rows than keys) times the split-KV forward
+(fa_fwd_splitkv: key-range pieces merged by their log-sum-exp, causal
+bottom-right aligned) instead; its line reports forward TFLOP/s.
 """
 from __future__ import annotations
 
@@ -37,9 +42,11 @@ NOMINAL_BF16_TFLOPS = 2250.0
 
 
 def flops(w):
-    f = 4.0 * w.B * w.Hq * w.Nq * w.Nk * w.d
-    if w.causal:
-        f /= 2
+    """Nominal FLOPs: 4*B*Hq*d per visible (query, key) pair, with Nq*Nk/2
+    pairs for causal Nq == Nk and Nq*Nk - Nq^2/2 for causal Nq < Nk
+    (bottom-right alignment)."""
+    pairs = w.Nq * w.Nk - (w.Nq * w.Nq / 2 if w.causal else 0)
+    f = 4.0 * w.B * w.Hq * pairs * w.d
     return f, 2.5 * f
 
 
@@ -54,7 +61,7 @@ def measured_peaks():
 
 
 def config_dict(w, n, l2_note):
-    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "Nq": w.Nq, "d": w.d,
             "causal": w.causal, "scale": "1/sqrt(d)", "global_batch": w.B * n, "seq_len": w.N,
             "parallelism": f"replicas x{n} (no collective: shards by batch/head)",
             "l2": l2_note}
@@ -299,6 +306,105 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(out), flush=True)
 
 
+def run_inference(args, rank, world, local_rank):
+    """Forward only, split-KV path, on an inference-shaped workload."""
+    import torch
+    import attn_inputs
+    import exact_io_aware_50_b200 as F
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = attn_inputs.BY_NAME[args.workload]
+    fwd_f, _ = flops(w)
+    x = attn_inputs.make(w, seed=w.seed + 1000 * rank)
+    g = {k: x[k].to(dev) for k in ("q", "k", "v")}
+    B, Hq, Hkv, Nq, Nk, d = w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d
+    splits = F.fa_fwd_splitkv_num_splits(B, Hq, Nq, Nk, d)
+    o = torch.empty_like(g["q"])
+    lse = torch.empty(B, Hq, Nq, device=dev, dtype=torch.float32)
+    ws = torch.empty(max(F.fa_fwd_splitkv_workspace_size(B, Hq, Nq, d, splits), 1), device=dev,
+                     dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        st = F.fa_fwd_splitkv(g["q"].data_ptr(), g["k"].data_ptr(), g["v"].data_ptr(),
+                              o.data_ptr(), lse.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                              w.scale, w.causal, splits, stream.cuda_stream)
+        if st != 0:
+            raise RuntimeError(f"fa_fwd_splitkv: {F.fa_strerror(st)}")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    if F.fa_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device error word set during the timed region")
+    total_ms = t0.elapsed_time(t1)
+    host = {k: x[k].pin_memory() for k in ("q", "k", "v")}
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + l_h.numel() * l_h.element_size()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(2, min(args.steps, 5))
+    a0.record(stream)
+    for _ in range(n_e2e):
+        for k2, t in host.items():
+            g[k2].copy_(t, non_blocking=True)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        l_h.copy_(lse, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1) / n_e2e
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
+    ms = total_ms / args.steps
+    burst, _, _, src = measured_peaks()
+    value = whole_job_tflops(world, fwd_f, ms)
+    out = {
+        "metric": "attention forward TFLOP/s (BF16, split-KV inference shape)",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
+        "config": dict(config_dict(w, world, "K/V 64 MiB (L2-resident between steps)"),
+                       num_splits=splits),
+        "roofline": {"bound": "tensor", "kernel": "fa_fwd_splitkv (pieces + merge)",
+                     "achieved": round(fwd_f / (ms * 1e-3) / 1e12, 2), "peak": burst,
+                     "peak_source": f"{src} bf16 dense burst (MEASURED_PEAKS.json)",
+                     "unit": "TFLOP/s", "frac": round(fwd_f / (ms * 1e-3) / 1e12 / burst, 4),
+                     "traffic": None},
+        "e2e": {"value": round(whole_job_tflops(world, fwd_f, e2e_ms), 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": (2 if splits > 1 else 1) * args.steps,
+        "clocks": clk,
+    }
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def load_traffic(workload, kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if
     one exists for this workload and the kernel source has not changed since
@@ -349,16 +455,18 @@ def cpu_baseline(w, seconds):
     heads = 0
     t0 = time.perf_counter()
     g = w.Hq // w.Hkv
+    off = w.Nk - w.Nq if w.causal else 0     # bottom-right alignment when Nq < Nk
     while True:
         h = heads % g
-        oracle.forward(q[:, h:h + 1], k, v, w.scale, w.causal)
-        oracle.backward(q[:, h:h + 1], k, v, do[:, h:h + 1], w.scale, w.causal)
+        oracle.forward(q[:, h:h + 1], k, v, w.scale, w.causal, off)
+        if w.backward:
+            oracle.backward(q[:, h:h + 1], k, v, do[:, h:h + 1], w.scale, w.causal)
         heads += 1
         el = time.perf_counter() - t0
         if el >= seconds or heads >= w.B * w.Hq:
             break
     fwd_f, bwd_f = flops(w)
-    per_head = (fwd_f + bwd_f) / (w.B * w.Hq)
+    per_head = (fwd_f + (bwd_f if w.backward else 0.0)) / (w.B * w.Hq)
     value = heads * per_head / el / 1e12
     cores = os.cpu_count()
     try:
@@ -369,7 +477,8 @@ def cpu_baseline(w, seconds):
     except Exception:
         pass
     return {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{heads} whole (batch 0, head) units of {w.name}, forward+backward, "
+            "sample": f"{heads} whole (batch 0, head) units of {w.name}, "
+                      f"{'forward+backward' if w.backward else 'forward'}, "
                       f"{el:.1f} s; full workload has {w.B * w.Hq} heads"}
 
 
@@ -417,8 +526,12 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
     if args.warmup < 3:
         args.warmup = 3
+    import attn_inputs
+    w = attn_inputs.BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif not w.backward and w.Nq < w.Nk:
+        run_inference(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

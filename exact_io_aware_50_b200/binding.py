@@ -24,7 +24,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libfa.so")
 _lib = None
 
-EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prep", "fa_bwd_dkdv",
+EXPORTS = ("fa_fwd", "fa_fwd_splitkv", "fa_fwd_splitkv_num_splits",
+           "fa_fwd_splitkv_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prep",
+           "fa_bwd_dkdv",
            "fa_bwd_dq", "fa_fwd_f32", "fa_bwd_f32", "fa_device_status", "fa_wait_selftest",
            "fa_exp2_eval", "fa_strerror")
 
@@ -49,6 +51,12 @@ def lib():
         L.fa_fwd.restype = I
         L.fa_fwd_f32.argtypes = [P] * 5 + dims
         L.fa_fwd_f32.restype = I
+        L.fa_fwd_splitkv.argtypes = [P] * 6 + [I, I, I, I, I, I, F, I, I, P]
+        L.fa_fwd_splitkv.restype = I
+        L.fa_fwd_splitkv_num_splits.argtypes = [I] * 5
+        L.fa_fwd_splitkv_num_splits.restype = I
+        L.fa_fwd_splitkv_workspace_size.argtypes = [I] * 5
+        L.fa_fwd_splitkv_workspace_size.restype = S
         L.fa_bwd.argtypes = [P] * 10 + dims
         L.fa_bwd.restype = I
         L.fa_bwd_f32.argtypes = [P] * 10 + dims
@@ -76,6 +84,20 @@ def lib():
 # ----------------------------------------------------------------- raw ABI
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
     return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, int(causal), stream)
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits,
+                   stream=0):
+    return lib().fa_fwd_splitkv(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, d, scale, int(causal),
+                                int(num_splits), stream)
+
+
+def fa_fwd_splitkv_num_splits(B, Hq, Nq, Nk, d):
+    return int(lib().fa_fwd_splitkv_num_splits(B, Hq, Nq, Nk, d))
+
+
+def fa_fwd_splitkv_workspace_size(B, Hq, Nq, d, num_splits):
+    return int(lib().fa_fwd_splitkv_workspace_size(B, Hq, Nq, d, num_splits))
 
 
 def fa_fwd_f32(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
@@ -164,6 +186,30 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
         raise ValueError("dtype must be bfloat16 or float32")
     _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), B, Hq, Hkv,
               Nq, Nk, d, scale, causal, _stream(q)), fn.__name__)
+    return o, L
+
+
+def forward_splitkv(q, k, v, scale=None, causal=False, num_splits=None, workspace=None):
+    """O, L for bf16 q [B, Hq, Nq, d] against k, v [B, Hkv, Nk, d] with the key
+    range cut into pieces merged by their log-sum-exp (fa_fwd_splitkv).
+    Causal is bottom-right aligned (Nq <= Nk).  num_splits=None picks
+    fa_fwd_splitkv_num_splits."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
+    scale = d ** -0.5 if scale is None else float(scale)
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("inputs must be contiguous bfloat16 CUDA tensors")
+    if num_splits is None:
+        num_splits = fa_fwd_splitkv_num_splits(B, Hq, Nq, Nk, d)
+    o = torch.empty_like(q)
+    L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(max(fa_fwd_splitkv_workspace_size(B, Hq, Nq, d, num_splits), 1),
+                                device=q.device, dtype=torch.uint8)
+    _check(fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                          workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits,
+                          _stream(q)), "fa_fwd_splitkv")
     return o, L
 
 

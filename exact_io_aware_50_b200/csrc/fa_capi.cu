@@ -44,11 +44,14 @@ int check_arch(int dev) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-int check_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal) {
+// bottom_right: causal with Nq <= Nk allowed (split-KV forward); otherwise
+// causal requires Nq == Nk.
+int check_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                bool bottom_right = false) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (causal && Nq != Nk) return FA_ERR_UNSUPPORTED;
+  if (causal && (bottom_right ? Nq > Nk : Nq != Nk)) return FA_ERR_UNSUPPORTED;
   // Tensor element counts must fit the kernels' index arithmetic.
   const double qe = (double)B * Hq * Nq * d, ke = (double)B * Hkv * Nk * d;
   if (qe > 4.0e12 || ke > 4.0e12) return FA_ERR_UNSUPPORTED;
@@ -131,7 +134,7 @@ FA_EXPORT const char *fa_strerror(int status) {
   switch (status) {
     case FA_OK: return "ok";
     case FA_ERR_INVALID_ARG: return "invalid argument (null pointer, size <= 0, Hq % Hkv != 0 or bad scale)";
-    case FA_ERR_UNSUPPORTED: return "unsupported configuration (head dim, causal with Nq != Nk, or size)";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration (head dim, causal query/key lengths, or size)";
     case FA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case FA_ERR_ARCH: return "device is not compute capability 10.0 (sm_100a build)";
     case FA_ERR_CUDA: return "CUDA runtime error or kernel launch failure";
@@ -161,6 +164,51 @@ FA_EXPORT int fa_fwd(const void *q, const void *k, const void *v, void *o, float
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.d = d;
   a.scale = scale; a.causal = causal ? 1 : 0; a.stream = (cudaStream_t)stream;
   return fa::launch_fwd_bf16_sm100(a);
+}
+
+FA_EXPORT int fa_fwd_splitkv_num_splits(int B, int Hq, int Nq, int Nk, int d) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0) return 0;
+  if (d != 64 && d != 128 && d != 256) return 0;
+  // Units of the plain forward (query blocks of 256 rows, 128 at d = 256);
+  // split the key range until about two waves of 148 SMs are busy, keeping
+  // at least two 128-key blocks per piece.
+  const long long rows_per_unit = d == 256 ? 128 : 256;
+  const long long units = (long long)B * Hq * ((Nq + rows_per_unit - 1) / rows_per_unit);
+  const long long kblocks = (Nk + 127) / 128;
+  long long s = (2 * 148 + units - 1) / units;
+  s = s < kblocks / 2 ? s : kblocks / 2;
+  s = s < 64 ? s : 64;
+  return s < 1 ? 1 : (int)s;
+}
+
+FA_EXPORT size_t fa_fwd_splitkv_workspace_size(int B, int Hq, int Nq, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0 || d <= 0 || num_splits <= 0) return 0;
+  if (num_splits == 1) return 0;
+  return fa::splitkv_ws_bytes(num_splits, B, Hq, Nq, d);
+}
+
+FA_EXPORT int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                             void *workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                             float scale, int causal, int num_splits, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (num_splits <= 0 || num_splits > 1024) return FA_ERR_INVALID_ARG;
+  if (num_splits > 1 && !workspace) return FA_ERR_INVALID_ARG;
+  int st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal, true);
+  if (st) return st;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!fa::aligned16(q) || !fa::aligned16(k) || !fa::aligned16(v) || !fa::aligned16(o) ||
+      !fa::aligned16(lse))
+    return FA_ERR_ALIGNMENT;
+  if (num_splits > 1 && ((uintptr_t)workspace & 255u)) return FA_ERR_ALIGNMENT;
+  AttnArgs a;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.ws = workspace;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.d = d;
+  a.scale = scale; a.causal = causal ? 1 : 0; a.stream = (cudaStream_t)stream;
+  a.causal_off = causal ? Nk - Nq : 0;
+  a.splits = num_splits;
+  return fa::launch_fwd_splitkv_bf16_sm100(a);
 }
 
 FA_EXPORT int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,

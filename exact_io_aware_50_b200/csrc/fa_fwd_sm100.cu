@@ -23,6 +23,15 @@
 //   warp  9    MMA issuer
 // The producer and MMA roles run in lane 0 alone (measured 6-8% faster on
 // B200 than keeping the warp converged around each wait).
+// Split-KV mode (inference shapes: few query blocks, long key range): work
+// unit = (piece, batch, head, query block); each piece covers a contiguous
+// range of the visible key blocks and writes its normalised partial output
+// (float32) and log-sum-exp to a workspace; splitkv_combine_kernel merges the
+// pieces with L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s, the
+// block-combination identity of the online softmax (blog section 2.2).  The
+// causal mask may be bottom-right aligned there (key j hidden from query i
+// when j > i + Nk - Nq).
+//
 // MMA issue order per block j (two tiles): PV0(j), S0(j+1), PV1(j), S1(j+1):
 // the softmax of one tile overlaps the tensor-core work of the other.
 // tcgen05 ops of one thread complete in issue order, and tcgen05.commit
@@ -83,6 +92,10 @@ struct FwdParams {
   int BH;            // B * Hq
   float scale_log2;  // scale * log2(e)
   int causal;
+  int causal_off;    // causal: key j hidden from query i when j > i + causal_off
+  int splits;        // pieces of the key range per query block (1: plain forward)
+  float *o_part;     // splits > 1: [splits][B*Hq][Nq][D] normalised partial O
+  float *l_part;     // splits > 1: [splits][B*Hq][Nq] partial log-sum-exp (natural log)
   unsigned *err;
 };
 
@@ -110,14 +123,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   // last wave holds the shortest units.  Otherwise all units cost the same and
   // they run head by head, so the K and V tiles a wave reads are those of a
   // few heads and stay in L2.
-  const int unit = blockIdx.x;
+  // Split-KV: the piece index is the slowest-varying part of the unit.
+  const int per_piece = p.nqb * p.BH;
+  const int piece = blockIdx.x / per_piece;
+  const int unit = blockIdx.x % per_piece;
   const int qblk = p.causal ? p.nqb - 1 - unit / p.BH : unit % p.nqb;
   const int bh = p.causal ? unit % p.BH : unit / p.nqb;
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int bh_kv = b * p.Hkv + h / (p.Hq / p.Hkv);
   const int q_start = qblk * C::NT * BM;
   const int nkb_all = (p.Nk + C::BN - 1) / C::BN;
-  const int nkb = p.causal ? min(nkb_all, (q_start + C::NT * BM + C::BN - 1) / C::BN) : nkb_all;
+  const int nkb_vis =
+      p.causal ? min(nkb_all, (q_start + C::NT * BM + p.causal_off + C::BN - 1) / C::BN) : nkb_all;
+  // key blocks [j0, j0 + nkb) of this piece
+  const int per_split = (nkb_vis + p.splits - 1) / p.splits;
+  const int j0 = min(nkb_vis, piece * per_split);
+  const int nkb = min(nkb_vis, j0 + per_split) - j0;
+  if (nkb == 0) {
+    // An empty piece (only in split mode): its rows see no key here.
+    for (int i = threadIdx.x; i < C::NT * BM; i += blockDim.x) {
+      const int row = q_start + i;
+      if (row >= p.Nq) break;
+      const size_t prow = ((size_t)piece * p.BH + bh) * p.Nq + row;
+      p.l_part[prow] = -INFINITY;
+      float4 *orow = reinterpret_cast<float4 *>(p.o_part + prow * C::D);
+      for (int e = 0; e < C::D / 4; ++e) orow[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -171,14 +204,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(B_KFULL + s), C::KV_TILE);
         for (int c = 0; c < C::DCH; ++c)
           tma_load_3d(sbase + C::OFF_K + s * C::KV_TILE + c * C::KV_CHUNK, &tmK, bar(B_KFULL + s),
-                      c * 64, j * C::BN, bh_kv);
+                      c * 64, (j0 + j) * C::BN, bh_kv);
         last_k_phase[s] = ph;
         ok = bounded_wait(bar(B_VEMPTY + s), ph ^ 1, wc);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(B_VFULL + s), C::KV_TILE);
         for (int c = 0; c < C::DCH; ++c)
           tma_load_3d(sbase + C::OFF_V + s * C::KV_TILE + c * C::KV_CHUNK, &tmV, bar(B_VFULL + s),
-                      c * 64, j * C::BN, bh_kv);
+                      c * 64, (j0 + j) * C::BN, bh_kv);
         last_v_phase[s] = ph;
       }
       if (!ok) {
@@ -274,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tP = tS + C::BN / 2;
     const uint32_t tO = tmem + lane_off + C::TM_O + t * C::D;
     const int row_lo = q_start + t * BM;
-    const int limit_row = p.causal ? min(p.Nk, row + 1) : p.Nk;  // keys [0, limit) visible
+    // keys [0, limit) visible
+    const int limit_row = p.causal ? min(p.Nk, row + 1 + p.causal_off) : p.Nk;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nkb; ++j) {
@@ -287,9 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
       float *s = reinterpret_cast<float *>(sr);
-      const int col_lo = j * C::BN;
+      const int col_lo = (j0 + j) * C::BN;
       const bool need_mask =
-          (col_lo + C::BN > p.Nk) || (p.causal && col_lo + C::BN - 1 > row_lo);
+          (col_lo + C::BN > p.Nk) || (p.causal && col_lo + C::BN - 1 > row_lo + p.causal_off);
       if (need_mask) {
         const int lim = limit_row - col_lo;
 #pragma unroll
@@ -352,7 +386,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------------------------------------------------- epilogue
     if (ok) ok = warp_wait_all(bar(B_OFULL + t), 0, wc);
-    if (ok) {
+    if (ok && p.splits > 1) {
+      // normalised partial output and log-sum-exp of this piece; a row whose
+      // keys in the piece are all hidden has l = 0: O_s = 0, L_s = -inf
+      tc_fence_after();
+      const bool empty = !(l_run > 0.f);
+      const float inv_l = empty ? 0.f : 1.f / l_run;
+      const bool live = row < p.Nq;
+      const size_t prow = ((size_t)piece * p.BH + bh) * p.Nq + (live ? row : 0);
+      float4 *orow = reinterpret_cast<float4 *>(p.o_part + prow * C::D);
+#pragma unroll 1
+      for (int c = 0; c < C::D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + c * 32, ov);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            orow[c * 8 + e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
+                                          __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                          __uint_as_float(ov[4 * e + 2]) * inv_l,
+                                          __uint_as_float(ov[4 * e + 3]) * inv_l);
+        }
+      }
+      if (live) p.l_part[prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    } else if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const bool live = row < p.Nq;
@@ -414,18 +472,80 @@ int run_fwd(const AttnArgs &a) {
   p.BH = a.B * a.Hq;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.causal = a.causal;
+  p.causal_off = a.causal_off;
+  p.splits = a.splits;
+  p.o_part = a.splits > 1 ? (float *)a.ws : nullptr;
+  p.l_part = a.splits > 1 ? (float *)((char *)a.ws + splitkv_l_offset(a.splits, a.B, a.Hq, a.Nq, a.d))
+                          : nullptr;
   p.err = a.err;
   auto kern = fwd_kernel<C>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return 5;
-  const long long units = (long long)p.nqb * p.BH;
+  const long long units = (long long)p.nqb * p.BH * p.splits;
   if (units > 2147483647LL) return 2;
   kern<<<(unsigned)units, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }
 
+// Merge the pieces of a split-KV forward, one warp per query row:
+// L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s -> bf16.
+template <int D>
+__global__ void splitkv_combine_kernel(const float *__restrict__ o_part,
+                                       const float *__restrict__ l_part, __nv_bfloat16 *__restrict__ o,
+                                       float *__restrict__ lse, int splits, long long rows) {
+  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float m = -INFINITY;
+  for (int s = 0; s < splits; ++s) m = fmaxf(m, l_part[(size_t)s * rows + row]);
+  constexpr int PER = D / 32;   // 2, 4 or 8 elements per lane
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float tot = 0.f;
+  if (m != -INFINITY) {
+    for (int s = 0; s < splits; ++s) {
+      const float ls = l_part[(size_t)s * rows + row];
+      if (ls == -INFINITY) continue;
+      const float w = __expf(ls - m);
+      tot += w;
+      const float *src = o_part + ((size_t)s * rows + row) * D + lane * PER;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+    }
+  }
+  const float inv = tot > 0.f ? 1.f / tot : 0.f;
+  __nv_bfloat16 *dst = o + row * D + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2)
+    *reinterpret_cast<uint32_t *>(dst + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+  if (lane == 0) lse[row] = tot > 0.f ? m + __logf(tot) : -INFINITY;
+}
+
+template <int D>
+int run_combine(const AttnArgs &a) {
+  const long long rows = (long long)a.B * a.Hq * a.Nq;
+  const float *o_part = (const float *)a.ws;
+  const float *l_part =
+      (const float *)((const char *)a.ws + splitkv_l_offset(a.splits, a.B, a.Hq, a.Nq, a.d));
+  splitkv_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, a.stream>>>(
+      o_part, l_part, (__nv_bfloat16 *)a.o, a.lse, a.splits, rows);
+  return cudaGetLastError() == cudaSuccess ? 0 : 5;
+}
+
 }  // namespace
+
+int launch_fwd_splitkv_bf16_sm100(const AttnArgs &a) {
+  int st = launch_fwd_bf16_sm100(a);
+  if (st || a.splits <= 1) return st;
+  switch (a.d) {
+    case 64: return run_combine<64>(a);
+    case 128: return run_combine<128>(a);
+    case 256: return run_combine<256>(a);
+    default: return 2;
+  }
+}
 
 int launch_fwd_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {

@@ -17,6 +17,8 @@ struct AttnArgs {
   int B = 0, Hq = 0, Hkv = 0, Nq = 0, Nk = 0, d = 0;
   float scale = 0.f;
   int causal = 0;
+  int causal_off = 0;           // causal: key j hidden from query i when j > i + causal_off
+  int splits = 1;               // split-KV forward: pieces of the key range (ws holds them)
   cudaStream_t stream = nullptr;
   unsigned *err = nullptr;      // device error word
 };
@@ -39,10 +41,21 @@ inline size_t ws_bytes(int B, int Hq, int Nq, int d) {
   return ws_dq_offset(B, Hq, Nq, d) + (size_t)B * Hq * Nq * d * 4;
 }
 
+// Split-KV forward workspace (float32): normalised partial outputs
+// [splits][B*Hq][Nq][d], then (256-byte aligned) partial log-sum-exps
+// [splits][B*Hq][Nq].
+inline size_t splitkv_l_offset(int splits, int B, int Hq, int Nq, int d) {
+  return ((size_t)splits * B * Hq * Nq * d * 4 + 255) & ~(size_t)255;
+}
+inline size_t splitkv_ws_bytes(int splits, int B, int Hq, int Nq, int d) {
+  return splitkv_l_offset(splits, B, Hq, Nq, d) + (size_t)splits * B * Hq * Nq * 4;
+}
+
 // Status codes use the fa_status numbering of fa.h.
 int launch_fwd_f32(const AttnArgs &a);
 int launch_bwd_f32(const AttnArgs &a);
 int launch_fwd_bf16_sm100(const AttnArgs &a);
+int launch_fwd_splitkv_bf16_sm100(const AttnArgs &a);   // pieces + merge (splits > 1)
 int launch_bwd_bf16_sm100(const AttnArgs &a);   // all three stages
 int launch_bwd_prep_bf16(const AttnArgs &a);     // D + zeroed dQ accumulator
 int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a);

@@ -71,6 +71,40 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
            fa_stream_t stream);
 
 /*
+ * Split-KV forward for inference shapes -- few query rows per head against a
+ * long key range (the FlashAttention blog, section 4.2, on batch-1 inference
+ * leaving the GPU idle when only batch and heads are parallel).  The visible
+ * key range of each 256-row query block (128 at d = 256) is cut into
+ * num_splits contiguous pieces of 128-key blocks, one CTA per piece; each
+ * piece's normalised output O_s (float32) and log-sum-exp L_s go to the
+ * workspace and a second kernel merges them:
+ *     L = log sum_s exp(L_s),   O = sum_s exp(L_s - L) O_s   -> bf16,
+ * the identity the online softmax uses to combine two blocks (blog section
+ * 2.2).  A piece that sees no key of a row has L_s = -inf and adds nothing.
+ *
+ * Causal here is bottom-right aligned: the Nq queries are the last Nq
+ * positions of the sequence, key j is hidden from query i when
+ * j > i + (Nk - Nq); Nq <= Nk is required (FA_ERR_UNSUPPORTED otherwise).
+ * For Nq == Nk this is fa_fwd's mask.
+ *
+ * fa_fwd_splitkv_num_splits -- a piece count that fills about two waves of
+ *   the GPU (0 for invalid sizes).
+ * fa_fwd_splitkv_workspace_size -- bytes of workspace for num_splits pieces:
+ *   float32 [num_splits][B][Hq][Nq][d] then, 256-byte aligned,
+ *   [num_splits][B][Hq][Nq]; 0 when num_splits == 1 (no workspace needed) or
+ *   a size is invalid.
+ * fa_fwd_splitkv -- tensors, dtypes and layouts as fa_fwd; workspace: at
+ *   least fa_fwd_splitkv_workspace_size(...) bytes, 256-byte aligned, may be
+ *   NULL when num_splits == 1; 1 <= num_splits <= 1024 (more pieces than key
+ *   blocks leave some empty), else FA_ERR_INVALID_ARG.
+ */
+int fa_fwd_splitkv_num_splits(int B, int Hq, int Nq, int Nk, int d);
+size_t fa_fwd_splitkv_workspace_size(int B, int Hq, int Nq, int d, int num_splits);
+int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                   void *workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                   int causal, int num_splits, fa_stream_t stream);
+
+/*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd and fa_bwd_f32
  * need (float32 throughout): the per-row vector D = rowsum(dO * O) and the
  * per-row base-2 log-sum-exp used by the backward, each padded to a multiple

@@ -104,3 +104,36 @@ def test_backward_argument_errors(fn):
 def test_selftest_rejects_bad_limit():
     assert F.fa_wait_selftest(0) == F.FA_ERR_INVALID_ARG
     assert F.fa_wait_selftest(2_000_000_000) == F.FA_ERR_INVALID_ARG
+
+
+def test_splitkv_argument_errors():
+    f = F.fa_fwd_splitkv
+
+    def call(ptrs=(FAKE,) * 6, Nq=8, Nk=16, d=64, causal=1, splits=2):
+        return f(*ptrs, 1, 2, 1, Nq, Nk, d, 0.125, causal, splits)
+
+    assert call(splits=0) == F.FA_ERR_INVALID_ARG
+    assert call(splits=2000) == F.FA_ERR_INVALID_ARG
+    assert call(ptrs=(FAKE,) * 5 + (0,)) == F.FA_ERR_INVALID_ARG   # workspace needed
+    assert call(ptrs=(0,) + (FAKE,) * 5) == F.FA_ERR_INVALID_ARG
+    assert call(Nq=17, Nk=16) == F.FA_ERR_UNSUPPORTED              # causal needs Nq <= Nk
+    assert call(d=96) == F.FA_ERR_UNSUPPORTED
+    assert call(ptrs=(FAKE,) * 5 + (FAKE + 16,)) == F.FA_ERR_ALIGNMENT   # workspace 256 B
+    assert call(ptrs=(FAKE + 4,) + (FAKE,) * 5) == F.FA_ERR_ALIGNMENT
+
+
+def test_splitkv_sizes():
+    def ws(B, H, N, d, s):
+        head = (s * B * H * N * d * 4 + 255) // 256 * 256
+        return head + s * B * H * N * 4
+    for (B, H, N, d, s) in ((1, 8, 512, 128, 19), (2, 3, 1000, 64, 7), (1, 1, 1, 256, 2)):
+        assert F.fa_fwd_splitkv_workspace_size(B, H, N, d, s) == ws(B, H, N, d, s)
+    assert F.fa_fwd_splitkv_workspace_size(1, 8, 512, 128, 1) == 0
+    assert F.fa_fwd_splitkv_workspace_size(1, 8, 512, 128, 0) == 0
+    # 16 units of 256 query rows -> ceil(2 * 148 / 16) = 19 pieces
+    assert F.fa_fwd_splitkv_num_splits(1, 8, 512, 16384, 128) == 19
+    # enough units already: one piece
+    assert F.fa_fwd_splitkv_num_splits(4, 16, 4096, 4096, 128) == 1
+    # capped at half the number of 128-key blocks
+    assert F.fa_fwd_splitkv_num_splits(1, 1, 1, 1024, 128) == 4
+    assert F.fa_fwd_splitkv_num_splits(0, 1, 1, 1024, 128) == 0
