@@ -37,6 +37,18 @@ What it computes (the plain definition, materialised, in float64):
   softmax of blog section 2.2 uses to combine two blocks' statistics:
       L = log sum_s exp(L_s),   O = sum_s exp(L_s - L) O_s.
   A piece that sees no key of a row has L_s = -inf and contributes nothing.
+* Dropout on P (the blog's section 5 call passes dropout_p to
+  F.scaled_dot_product_attention; the pages use 0).  Reading adopted: inverted
+  dropout of the normalised probabilities, O = (P * Z) V / (1 - p) with
+  Z_ij in {0, 1}, while L stays the log-sum-exp of the undropped scores.  The
+  mask is a pure function of (seed, offset, batch*Hq + head, i, j): the
+  counter-based generator Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
+  "Parallel random numbers: as easy as 1, 2, 3", SC 2011) with key
+  (seed mod 2^32, seed >> 32) and counter (j >> 2, i, b*Hq + h, offset mod
+  2^32); output word j mod 4 is compared with floor(p * 2^32) and the element
+  is kept when the word is not smaller.  Backward of f = sum(O * dO):
+      dV = (P*Z)^T dO / (1-p),  dP = (dO V^T) * Z / (1-p),
+      D_i = sum_j P_ij dP_ij (= sum_d dO_id O_id),  dS = P * (dP - D).
 * Block-wise forms -- the online-softmax step of blog section 2.2 (normalise at
   every block, "v1") and the deferred-normalisation loop of blog section 4.1
   and the CSDN tutorial section 3 ("v2": keep O unnormalised, rescale by
@@ -67,6 +79,13 @@ __all__ = [
     "blockwise_forward_v2",
     "merge_partials",
     "splitkv_forward",
+    "philox4x32_10",
+    "dropout_keep",
+    "dropout_forward",
+    "dropout_backward",
+    "dropout_forward_rows",
+    "dropout_backward_rows",
+    "dropout_backward_kv_rows",
 ]
 
 
@@ -354,3 +373,139 @@ def splitkv_forward(q, k, v, scale, causal, bounds, causal_offset=0):
                 lse_parts[p_, b, h] = lp
     o, lse = merge_partials(o_parts, lse_parts)
     return o, lse, o_parts, lse_parts
+
+
+# ---------------------------------------------------------------------------
+# Dropout: Philox4x32-10 mask, forward and backward with the mask applied.
+# ---------------------------------------------------------------------------
+
+_PHILOX_M = (0xD2511F53, 0xCD9E8D57)      # round multipliers
+_PHILOX_W = (0x9E3779B9, 0xBB67AE85)      # key increments (golden ratio, sqrt(3) - 1)
+_U32 = np.uint64(0xFFFFFFFF)
+
+
+def philox4x32_10(c0, c1, c2, c3, k0, k1):
+    """Philox4x32 with 10 rounds, elementwise over arrays of 32-bit counters.
+
+    One round maps (c0, c1, c2, c3) to
+        (hi(M1*c2) ^ c1 ^ k0, lo(M1*c2), hi(M0*c0) ^ c3 ^ k1, lo(M0*c0))
+    and the key is then advanced by (W0, W1) modulo 2^32.  Returns the four
+    output words as uint64 arrays holding 32-bit values."""
+    c = [np.asarray(x, dtype=np.uint64) & _U32 for x in (c0, c1, c2, c3)]
+    k0 = np.uint64(int(k0) & 0xFFFFFFFF)
+    k1 = np.uint64(int(k1) & 0xFFFFFFFF)
+    m0, m1 = np.uint64(_PHILOX_M[0]), np.uint64(_PHILOX_M[1])
+    for _ in range(10):
+        p0 = m0 * c[0]
+        p1 = m1 * c[2]
+        c = [((p1 >> np.uint64(32)) ^ c[1] ^ k0) & _U32, p1 & _U32,
+             ((p0 >> np.uint64(32)) ^ c[3] ^ k1) & _U32, p0 & _U32]
+        k0 = (k0 + np.uint64(_PHILOX_W[0])) & _U32
+        k1 = (k1 + np.uint64(_PHILOX_W[1])) & _U32
+    return c
+
+
+def dropout_keep(bh, rows, cols, p, seed, offset):
+    """Keep mask Z [len(rows), len(cols)] of head index bh = b*Hq + h."""
+    rows = np.asarray(rows, dtype=np.uint64)[:, None]
+    cols = np.asarray(cols, dtype=np.uint64)[None, :]
+    words = philox4x32_10(cols >> np.uint64(2), rows, np.uint64(bh), np.uint64(int(offset) & 0xFFFFFFFF),
+                          int(seed) & 0xFFFFFFFF, int(seed) >> 32)
+    pick = (cols & np.uint64(3)) + np.zeros_like(rows)
+    w = np.choose(pick.astype(np.int64), words)
+    thr = np.uint64(int(np.floor(np.float64(p) * 4294967296.0)))
+    return w >= thr
+
+
+def _head_probs(q2, k2, scale, causal, rows=None, causal_offset=0):
+    if rows is None:
+        s = scores(q2, k2, scale, causal, causal_offset)
+    else:
+        s = _row_chunk_scores(q2, k2, scale, causal, rows, causal_offset)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = np.sum(e, axis=1, keepdims=True)
+    return e / l, (m + np.log(l))[:, 0]
+
+
+def dropout_forward(q, k, v, scale, causal, p, seed, offset):
+    """O = (P * Z) V / (1 - p), L = logsumexp of the undropped scores."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    o = np.empty((B, Hq, Nq, v.shape[3]))
+    lse = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            kh = _kv_head(h, Hq, Hkv)
+            pr, lse[b, h] = _head_probs(q[b, h], k[b, kh], scale, causal)
+            z = dropout_keep(b * Hq + h, np.arange(Nq), np.arange(Nk), p, seed, offset)
+            o[b, h] = (pr * z) @ v[b, kh] / (1.0 - p)
+    return o, lse
+
+
+def dropout_backward(q, k, v, do, scale, causal, p, seed, offset):
+    """Gradients of f = sum(O * dO) for dropout_forward; returns (dq, dk, dv, D)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dsum = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            kh = _kv_head(h, Hq, Hkv)
+            pr, _ = _head_probs(q[b, h], k[b, kh], scale, causal)
+            z = dropout_keep(b * Hq + h, np.arange(Nq), np.arange(Nk), p, seed, offset)
+            dv[b, kh] += (pr * z).T @ do[b, h] / (1.0 - p)
+            dp = (do[b, h] @ v[b, kh].T) * z / (1.0 - p)
+            D = np.sum(pr * dp, axis=1)
+            ds = pr * (dp - D[:, None])
+            dq[b, h] = scale * (ds @ k[b, kh])
+            dk[b, kh] += scale * (ds.T @ q[b, h])
+            dsum[b, h] = D
+    return dq, dk, dv, dsum
+
+
+def dropout_forward_rows(q2, k2, v2, scale, causal, rows, bh, p, seed, offset):
+    """dropout_forward for chosen query rows of one head (bh = b*Hq + h)."""
+    rows = np.asarray(rows)
+    pr, lse = _head_probs(_f64(q2), _f64(k2), scale, causal, rows)
+    z = dropout_keep(bh, rows, np.arange(k2.shape[0]), p, seed, offset)
+    return (pr * z) @ _f64(v2) / (1.0 - p), lse
+
+
+def dropout_backward_rows(q2, k2, v2, do2, scale, causal, rows, bh, p, seed, offset):
+    """dQ and D for chosen query rows of one head (dropout)."""
+    rows = np.asarray(rows)
+    pr, _ = _head_probs(_f64(q2), _f64(k2), scale, causal, rows)
+    z = dropout_keep(bh, rows, np.arange(k2.shape[0]), p, seed, offset)
+    dp = (_f64(do2)[rows] @ _f64(v2).T) * z / (1.0 - p)
+    D = np.sum(pr * dp, axis=1)
+    ds = pr * (dp - D[:, None])
+    return scale * (ds @ _f64(k2)), D
+
+
+def dropout_backward_kv_rows(q_heads, k2, v2, do_heads, bhs, scale, causal, kv_rows, p, seed,
+                             offset, chunk=2048):
+    """dK and dV for chosen key rows of one key/value head (dropout); bhs are
+    the b*Hq + h indices of the query heads in q_heads."""
+    kv_rows = np.asarray(kv_rows)
+    k2, v2 = _f64(k2), _f64(v2)
+    dk = np.zeros((len(kv_rows), k2.shape[1]))
+    dv = np.zeros((len(kv_rows), v2.shape[1]))
+    for q2, do2, bh in zip(q_heads, do_heads, bhs):
+        q2, do2 = _f64(q2), _f64(do2)
+        nq = q2.shape[0]
+        for c in range(0, nq, chunk):
+            r = np.arange(c, min(c + chunk, nq))
+            pr, _ = _head_probs(q2, k2, scale, causal, r)
+            z = dropout_keep(bh, r, np.arange(k2.shape[0]), p, seed, offset)
+            dp = (do2[r] @ v2.T) * z / (1.0 - p)
+            D = np.sum(pr * dp, axis=1)
+            pj, zj = pr[:, kv_rows], z[:, kv_rows]
+            dsj = pj * (dp[:, kv_rows] - D[:, None])
+            dv += (pj * zj).T @ do2[r] / (1.0 - p)
+            dk += scale * (dsj.T @ q2[r])
+    return dk, dv
