@@ -24,7 +24,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libfa.so")
 _lib = None
 
-EXPORTS = ("fa_fwd", "fa_fwd_splitkv", "fa_fwd_splitkv_num_splits",
+EXPORTS = ("fa_fwd", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_splitkv",
+           "fa_fwd_splitkv_num_splits",
            "fa_fwd_splitkv_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prep",
            "fa_bwd_dkdv",
            "fa_bwd_dq", "fa_fwd_f32", "fa_bwd_f32", "fa_device_status", "fa_wait_selftest",
@@ -51,6 +52,11 @@ def lib():
         L.fa_fwd.restype = I
         L.fa_fwd_f32.argtypes = [P] * 5 + dims
         L.fa_fwd_f32.restype = I
+        U64 = ctypes.c_ulonglong
+        L.fa_fwd_dropout.argtypes = [P] * 5 + [I, I, I, I, I, I, F, I, F, U64, U64, P]
+        L.fa_fwd_dropout.restype = I
+        L.fa_bwd_dropout.argtypes = [P] * 10 + [I, I, I, I, I, I, F, I, F, U64, U64, P]
+        L.fa_bwd_dropout.restype = I
         L.fa_fwd_splitkv.argtypes = [P] * 6 + [I, I, I, I, I, I, F, I, I, P]
         L.fa_fwd_splitkv.restype = I
         L.fa_fwd_splitkv_num_splits.argtypes = [I] * 5
@@ -84,6 +90,18 @@ def lib():
 # ----------------------------------------------------------------- raw ABI
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
     return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, int(causal), stream)
+
+
+def fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, p_drop, seed, offset,
+                   stream=0):
+    return lib().fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, int(causal),
+                                float(p_drop), int(seed), int(offset), stream)
+
+
+def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                   p_drop, seed, offset, stream=0):
+    return lib().fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, ws, B, Hq, Hkv, Nq, Nk, d,
+                                scale, int(causal), float(p_drop), int(seed), int(offset), stream)
 
 
 def fa_fwd_splitkv(q, k, v, o, lse, ws, B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits,
@@ -211,6 +229,39 @@ def forward_splitkv(q, k, v, scale=None, causal=False, num_splits=None, workspac
                           workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits,
                           _stream(q)), "fa_fwd_splitkv")
     return o, L
+
+
+def forward_dropout(q, k, v, p_drop, seed, offset=0, scale=None, causal=False):
+    """O, L with dropout on P (bf16, fa_fwd_dropout)."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
+    scale = d ** -0.5 if scale is None else float(scale)
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("inputs must be contiguous bfloat16 CUDA tensors")
+    o = torch.empty_like(q)
+    L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
+    _check(fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                          B, Hq, Hkv, Nq, Nk, d, scale, causal, p_drop, seed, offset, _stream(q)),
+           "fa_fwd_dropout")
+    return o, L
+
+
+def backward_dropout(q, k, v, o, lse, dout, p_drop, seed, offset=0, scale=None, causal=False,
+                     workspace=None):
+    """dQ, dK, dV of forward_dropout with the same seed and offset."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
+    scale = d ** -0.5 if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_size(B, Hq, Nq, d), device=q.device,
+                                dtype=torch.uint8)
+    _check(fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, p_drop, seed,
+                          offset, _stream(q)), "fa_bwd_dropout")
+    return dq, dk, dv
 
 
 def backward(q, k, v, o, lse, dout, scale=None, causal=False, workspace=None):

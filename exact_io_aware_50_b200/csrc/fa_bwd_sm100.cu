@@ -140,8 +140,34 @@ struct BwdParams {
   int Hq, Hkv, Nq, Nk, npad, nqb, nkb, BHkv;
   float scale, scale_log2;
   int causal;
+  // dropout on P (wide kernel, DROP instances): keep when the Philox word is
+  // >= drop_thr; dV and dP are scaled by drop_scale = 1 / (1 - p)
+  uint32_t drop_thr, seed_lo, seed_hi, drop_off;
+  float drop_scale;
   unsigned *err;
 };
+
+// Keep bits of the dropout mask for key row kv (this thread) and the four
+// query columns i0 .. i0 + 3 (bit c for column i0 + c).  The four threads of
+// a lane quad hold four consecutive key rows, which share one Philox counter
+// (kv / 4, i): thread l of the quad evaluates the counter of column i0 + l
+// and the quad exchanges words so that each thread gets word kv % 4 of all
+// four columns.  All 32 lanes must call this together.
+__device__ __forceinline__ uint32_t dropout_keep4(int kv, int i0, uint32_t bhq, const BwdParams &p,
+                                                  int lane) {
+  const int l = lane & 3;
+  const uint4 R = philox4x32_10((uint32_t)kv >> 2, (uint32_t)(i0 + l), bhq, p.drop_off, p.seed_lo,
+                                p.seed_hi);
+  auto word = [&](int idx) { return idx == 0 ? R.x : idx == 1 ? R.y : idx == 2 ? R.z : R.w; };
+  uint32_t bits = (word(l) >= p.drop_thr) ? (1u << l) : 0u;
+#pragma unroll
+  for (int k = 1; k < 4; ++k) {
+    // lane l reads from quad lane s = l + k the word s sent, word (s - k) = l
+    const uint32_t got = __shfl_sync(0xffffffffu, word((l - k) & 3), (lane & ~3) | ((l + k) & 3));
+    bits |= (got >= p.drop_thr) ? (1u << ((l + k) & 3)) : 0u;
+  }
+  return bits;
+}
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
                                           uint32_t bar) {
@@ -682,7 +708,7 @@ struct BwdWideCfg {
   static_assert(D == 64 || D == 128, "wide path is for d = 64 and 128");
 };
 
-template <class C>
+template <class C, bool DROP>
 __global__ void __launch_bounds__(C::THREADS, 1)
     bwd_wide_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -933,6 +959,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_fence_after();
       // ---- phase 1: P^T for query columns [64 wg, 64 wg + 64), 16 at a time
       uint32_t pkeep[4][8];
+      uint32_t keepbits[2] = {0u, 0u};               // dropout: bit c = column 64 wg + c kept
+      const uint32_t bhq = (uint32_t)(b * p.Hq + step_head(i));
 #pragma unroll
       for (int sb = 0; sb < 4; ++sb) {
         const int c0 = 64 * wg + 16 * sb;
@@ -959,8 +987,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) pkeep[sb][e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
         // P^T of query columns 32h + 16(sb%2) + [0,16) -> A columns 32h + 8(sb%2) + [0,8),
-        // all of which this thread has already read
-        tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 8 * (sb & 1), pkeep[sb]);
+        // all of which this thread has already read.  With dropout the dV
+        // operand is P^T * Z; pkeep keeps P^T for dS.
+        if (DROP) {
+          uint32_t m16 = 0;
+#pragma unroll
+          for (int gq = 0; gq < 4; ++gq)
+            m16 |= dropout_keep4(kv, q0 + c0 + 4 * gq, bhq, p, lane) << (4 * gq);
+          keepbits[sb >> 1] |= m16 << (16 * (sb & 1));
+          uint32_t pm[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            pm[e] = pack_bf16x2(((m16 >> (2 * e)) & 1u) ? pr[2 * e] : 0.f,
+                                ((m16 >> (2 * e + 1)) & 1u) ? pr[2 * e + 1] : 0.f);
+          tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 8 * (sb & 1), pm);
+        } else {
+          tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 8 * (sb & 1), pkeep[sb]);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -987,7 +1030,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int c = 4 * e4 + u;
             const uint32_t pp = pkeep[sb][c >> 1];
             const float pv = __uint_as_float((c & 1) ? (pp & 0xffff0000u) : (pp << 16));
-            ds[u] = pv * (__uint_as_float(dv[c]) - dd[u]);
+            float dpv = __uint_as_float(dv[c]);
+            if (DROP) dpv = ((keepbits[sb >> 1] >> (16 * (sb & 1) + c)) & 1u) ? dpv * p.drop_scale : 0.f;
+            ds[u] = pv * (dpv - dd[u]);
           }
           dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
           dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
@@ -1016,7 +1061,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const size_t rowoff = ((size_t)bhkv * p.Nk + (kv_live ? kv : 0)) * C::D;
       const uint32_t src = tmem + lane_off + (wg ? C::TM_DK : C::TM_DV);
       __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + rowoff;
-      const float mul = wg ? p.scale : 1.f;
+      const float mul = wg ? p.scale : (DROP ? p.drop_scale : 1.f);
 #pragma unroll 1
       for (int c = 0; c < C::D / 32; ++c) {
         uint32_t v[32];
@@ -1224,13 +1269,19 @@ int run_dkdv(const AttnArgs &a) {
   p.err = a.err;
   const long long units = (long long)p.nkb * p.BHkv;
   if (units > 2147483647LL) return 2;
+  p.drop_thr = a.drop_thr;
+  p.seed_lo = (uint32_t)a.seed;
+  p.seed_hi = (uint32_t)(a.seed >> 32);
+  p.drop_off = (uint32_t)a.drop_offset;
+  p.drop_scale = a.drop_scale;
   if constexpr (WIDE) {
-    auto kern = bwd_wide_kernel<C>;
+    auto kern = a.drop_thr != 0 ? bwd_wide_kernel<C, true> : bwd_wide_kernel<C, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
       return 5;
     kern<<<(unsigned)units, C::THREADS, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
   } else {
+    if (a.drop_thr != 0) return 2;   // dropout runs in the wide kernel only (d <= 128)
     auto kern = bwd_kernel<C>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)

@@ -60,6 +60,18 @@ int check_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int 
   return FA_OK;
 }
 
+// Dropout probability -> keep threshold floor(p * 2^32) and 1 / (1 - p);
+// FA_ERR_INVALID_ARG unless 0 <= p < 1.
+int dropout_params(float p_drop, unsigned long long seed, unsigned long long offset, AttnArgs &a) {
+  if (!(p_drop >= 0.f) || !(p_drop < 1.f)) return FA_ERR_INVALID_ARG;
+  const double t = floor((double)p_drop * 4294967296.0);
+  a.drop_thr = t >= 4294967295.0 ? 0xFFFFFFFFu : (uint32_t)t;
+  a.drop_scale = (float)(1.0 / (1.0 - (double)p_drop));
+  a.seed = seed;
+  a.drop_offset = offset;
+  return FA_OK;
+}
+
 int prologue(int *dev, AttnArgs &a) {
   int st = current_device_checked(dev);
   if (st) return st;
@@ -170,12 +182,14 @@ FA_EXPORT int fa_fwd_splitkv_num_splits(int B, int Hq, int Nq, int Nk, int d) {
   if (B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0) return 0;
   if (d != 64 && d != 128 && d != 256) return 0;
   // Units of the plain forward (query blocks of 256 rows, 128 at d = 256);
-  // split the key range until about two waves of 148 SMs are busy, keeping
-  // at least two 128-key blocks per piece.
+  // split the key range so that one wave of 148 SMs is as full as it gets
+  // without a second, partial wave (measured best on B200: B1 H8 Nq512
+  // Nk16384 d128 runs 52 us with 9 pieces, 67 us with 19), keeping at least
+  // two 128-key blocks per piece.
   const long long rows_per_unit = d == 256 ? 128 : 256;
   const long long units = (long long)B * Hq * ((Nq + rows_per_unit - 1) / rows_per_unit);
   const long long kblocks = (Nk + 127) / 128;
-  long long s = (2 * 148 + units - 1) / units;
+  long long s = 148 / units;
   s = s < kblocks / 2 ? s : kblocks / 2;
   s = s < 64 ? s : 64;
   return s < 1 ? 1 : (int)s;
@@ -224,6 +238,52 @@ FA_EXPORT int fa_bwd(const void *q, const void *k, const void *v, const void *o,
     if (!fa::aligned16(p)) return FA_ERR_ALIGNMENT;
   if (((uintptr_t)workspace & 255u) != 0) return FA_ERR_ALIGNMENT;
   AttnArgs a;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.q = q; a.k = k; a.v = v; a.o_in = o; a.lse = const_cast<float *>(lse); a.dout = dout;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.ws = workspace;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.d = d;
+  a.scale = scale; a.causal = causal ? 1 : 0; a.stream = (cudaStream_t)stream;
+  return fa::launch_bwd_bf16_sm100(a);
+}
+
+FA_EXPORT int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse,
+                             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                             float p_drop, unsigned long long seed, unsigned long long offset,
+                             fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  AttnArgs a;
+  int st = fa::dropout_params(p_drop, seed, offset, a);
+  if (st) return st;
+  if ((st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal))) return st;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!fa::aligned16(q) || !fa::aligned16(k) || !fa::aligned16(v) || !fa::aligned16(o) ||
+      !fa::aligned16(lse))
+    return FA_ERR_ALIGNMENT;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.d = d;
+  a.scale = scale; a.causal = causal ? 1 : 0; a.stream = (cudaStream_t)stream;
+  return fa::launch_fwd_bf16_sm100(a);
+}
+
+FA_EXPORT int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o,
+                             const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                             void *workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                             float scale, int causal, float p_drop, unsigned long long seed,
+                             unsigned long long offset, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return FA_ERR_INVALID_ARG;
+  AttnArgs a;
+  int st = fa::dropout_params(p_drop, seed, offset, a);
+  if (st) return st;
+  if ((st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal))) return st;
+  if (d != 64 && d != 128 && !(d == 256 && a.drop_thr == 0)) return FA_ERR_UNSUPPORTED;
+  const void *ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+  for (const void *p : ptrs)
+    if (!fa::aligned16(p)) return FA_ERR_ALIGNMENT;
+  if (((uintptr_t)workspace & 255u) != 0) return FA_ERR_ALIGNMENT;
   int dev;
   if ((st = fa::prologue(&dev, a))) return st;
   a.q = q; a.k = k; a.v = v; a.o_in = o; a.lse = const_cast<float *>(lse); a.dout = dout;

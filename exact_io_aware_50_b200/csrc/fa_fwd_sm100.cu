@@ -96,10 +96,14 @@ struct FwdParams {
   int splits;        // pieces of the key range per query block (1: plain forward)
   float *o_part;     // splits > 1: [splits][B*Hq][Nq][D] normalised partial O
   float *l_part;     // splits > 1: [splits][B*Hq][Nq] partial log-sum-exp (natural log)
+  // dropout on P (DROP kernels): keep when the Philox word >= drop_thr; kept
+  // values are scaled by drop_scale = 1 / (1 - p) in the epilogue
+  uint32_t drop_thr, seed_lo, seed_hi, drop_off;
+  float drop_scale;
   unsigned *err;
 };
 
-template <class C>
+template <class C, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -350,12 +354,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // p = 2^(s * scale * log2e - m): one column in four on the FMA pipe
-      // (exp2_poly), the rest on MUFU; row sum in four independent partials
+      // p = 2^(s * scale * log2e - m) on MUFU (exp2_poly for one column in
+      // four when FA_FWD_POLY_EXP is set); row sum in four independent
+      // partials over the undropped p; with dropout, P in TMEM keeps only the
+      // columns whose Philox word is >= drop_thr (one Philox call per four
+      // key columns)
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < C::BN / 32; ++c) {
         uint32_t pk[16];
+        uint4 rnd = make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float x0 = fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_use);
@@ -363,7 +371,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float p0 = fast_exp2(x0);
           const float p1 = (kPolyExp && (e & 1)) ? exp2_poly(x1) : fast_exp2(x1);
           rs[e & 3] += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          if (DROP) {
+            if ((e & 1) == 0)
+              rnd = philox4x32_10((uint32_t)(col_lo + c * 32 + 2 * e) >> 2, (uint32_t)row,
+                                  (uint32_t)bh, p.drop_off, p.seed_lo, p.seed_hi);
+            const uint32_t w0 = (e & 1) ? rnd.z : rnd.x, w1 = (e & 1) ? rnd.w : rnd.y;
+            pk[e] = pack_bf16x2(w0 >= p.drop_thr ? p0 : 0.f, w1 >= p.drop_thr ? p1 : 0.f);
+          } else {
+            pk[e] = pack_bf16x2(p0, p1);
+          }
         }
         tmem_st16(tP + c * 16, pk);
       }
@@ -412,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (live) p.l_part[prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
     } else if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l_run;
+      const float inv_l = (DROP ? p.drop_scale : 1.f) / l_run;
       const bool live = row < p.Nq;
       __nv_bfloat16 *orow = p.o + ((size_t)bh * p.Nq + (live ? row : 0)) * C::D;
 #pragma unroll 1
@@ -477,8 +493,14 @@ int run_fwd(const AttnArgs &a) {
   p.o_part = a.splits > 1 ? (float *)a.ws : nullptr;
   p.l_part = a.splits > 1 ? (float *)((char *)a.ws + splitkv_l_offset(a.splits, a.B, a.Hq, a.Nq, a.d))
                           : nullptr;
+  p.drop_thr = a.drop_thr;
+  p.seed_lo = (uint32_t)a.seed;
+  p.seed_hi = (uint32_t)(a.seed >> 32);
+  p.drop_off = (uint32_t)a.drop_offset;
+  p.drop_scale = a.drop_scale;
   p.err = a.err;
-  auto kern = fwd_kernel<C>;
+  if (a.drop_thr != 0 && a.splits > 1) return 2;   // dropout only in the plain forward
+  auto kern = a.drop_thr != 0 ? fwd_kernel<C, true> : fwd_kernel<C, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return 5;

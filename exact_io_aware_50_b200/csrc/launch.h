@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 namespace fa {
 
@@ -19,6 +20,12 @@ struct AttnArgs {
   int causal = 0;
   int causal_off = 0;           // causal: key j hidden from query i when j > i + causal_off
   int splits = 1;               // split-KV forward: pieces of the key range (ws holds them)
+  // dropout on P: keep element (b, h, i, j) when word j % 4 of
+  // Philox4x32-10(key = seed, counter = (j / 4, i, b*Hq + h, offset)) is
+  // >= drop_thr = floor(p * 2^32); 0 = no dropout.  drop_scale = 1 / (1 - p).
+  uint32_t drop_thr = 0;
+  float drop_scale = 1.f;
+  unsigned long long seed = 0, drop_offset = 0;
   cudaStream_t stream = nullptr;
   unsigned *err = nullptr;      // device error word
 };

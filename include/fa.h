@@ -87,8 +87,8 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
  * j > i + (Nk - Nq); Nq <= Nk is required (FA_ERR_UNSUPPORTED otherwise).
  * For Nq == Nk this is fa_fwd's mask.
  *
- * fa_fwd_splitkv_num_splits -- a piece count that fills about two waves of
- *   the GPU (0 for invalid sizes).
+ * fa_fwd_splitkv_num_splits -- a piece count that fills one wave of the
+ *   GPU's 148 SMs (1 when the query blocks alone do; 0 for invalid sizes).
  * fa_fwd_splitkv_workspace_size -- bytes of workspace for num_splits pieces:
  *   float32 [num_splits][B][Hq][Nq][d] then, 256-byte aligned,
  *   [num_splits][B][Hq][Nq]; 0 when num_splits == 1 (no workspace needed) or
@@ -103,6 +103,35 @@ size_t fa_fwd_splitkv_workspace_size(int B, int Hq, int Nq, int d, int num_split
 int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
                    void *workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
                    int causal, int num_splits, fa_stream_t stream);
+
+/*
+ * Dropout on P (BF16).  The blog's section 5 call passes dropout_p to
+ * F.scaled_dot_product_attention (0 there); these entry points take p > 0:
+ *     O = (P * Z) V / (1 - p),   L = log-sum-exp of the undropped scores,
+ * with Z_ij = 1 when word (j mod 4) of Philox4x32-10 (Salmon et al.,
+ * "Parallel random numbers: as easy as 1, 2, 3", SC 2011) with
+ *     key     = (seed mod 2^32, seed >> 32),
+ *     counter = (j / 4, i, b*Hq + h, offset mod 2^32)
+ * is >= floor(p * 2^32), else 0 (i query row, j key column, h query head).
+ * The mask is a pure function of (seed, offset, b, h, i, j): fa_bwd_dropout
+ * with the same seed and offset regenerates it.  Gradients of
+ * f = sum(O * dO): dV = (P*Z)^T dO / (1-p), dP = (dO V^T) * Z / (1-p),
+ * dS = P * (dP - D) with D = rowsum(dO * O).
+ *
+ * Same tensors, layouts, size rules and errors as fa_fwd / fa_bwd, plus:
+ * 0 <= p_drop < 1 (else FA_ERR_INVALID_ARG); p_drop = 0 computes exactly
+ * fa_fwd / fa_bwd.  fa_bwd_dropout with p_drop > 0 supports d = 64 and 128
+ * (FA_ERR_UNSUPPORTED for d = 256).
+ */
+int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   float p_drop, unsigned long long seed, unsigned long long offset,
+                   fa_stream_t stream);
+int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                   const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   float p_drop, unsigned long long seed, unsigned long long offset,
+                   fa_stream_t stream);
 
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd and fa_bwd_f32

@@ -130,10 +130,26 @@ def test_splitkv_sizes():
         assert F.fa_fwd_splitkv_workspace_size(B, H, N, d, s) == ws(B, H, N, d, s)
     assert F.fa_fwd_splitkv_workspace_size(1, 8, 512, 128, 1) == 0
     assert F.fa_fwd_splitkv_workspace_size(1, 8, 512, 128, 0) == 0
-    # 16 units of 256 query rows -> ceil(2 * 148 / 16) = 19 pieces
-    assert F.fa_fwd_splitkv_num_splits(1, 8, 512, 16384, 128) == 19
+    # 16 units of 256 query rows -> floor(148 / 16) = 9 pieces (one wave)
+    assert F.fa_fwd_splitkv_num_splits(1, 8, 512, 16384, 128) == 9
     # enough units already: one piece
     assert F.fa_fwd_splitkv_num_splits(4, 16, 4096, 4096, 128) == 1
     # capped at half the number of 128-key blocks
     assert F.fa_fwd_splitkv_num_splits(1, 1, 1, 1024, 128) == 4
     assert F.fa_fwd_splitkv_num_splits(0, 1, 1, 1024, 128) == 0
+
+
+def test_dropout_argument_errors():
+    def fwd(p, d=64, ptrs=(FAKE,) * 5):
+        return F.fa_fwd_dropout(*ptrs, 1, 2, 1, 8, 8, d, 0.125, 0, p, 1, 0)
+
+    def bwd(p, d=64):
+        return F.fa_bwd_dropout(*(FAKE,) * 10, 1, 2, 1, 8, 8, d, 0.125, 0, p, 1, 0)
+
+    for bad in (-0.1, 1.0, 1.5, float("nan")):
+        assert fwd(bad) == F.FA_ERR_INVALID_ARG
+        assert bwd(bad) == F.FA_ERR_INVALID_ARG
+    assert fwd(0.1, ptrs=(0,) + (FAKE,) * 4) == F.FA_ERR_INVALID_ARG
+    assert fwd(0.1, d=96) == F.FA_ERR_UNSUPPORTED
+    assert bwd(0.1, d=256) == F.FA_ERR_UNSUPPORTED      # dropout backward: d = 64, 128
+    assert fwd(0.1, ptrs=(FAKE + 2,) + (FAKE,) * 4) == F.FA_ERR_ALIGNMENT
