@@ -24,23 +24,24 @@
 //             padded to 128-row blocks, and the zeroed f32 dQ accumulator;
 //   dkdv   one CTA per (batch, key/value head, 128-row key block); K - c and
 //          V stay in shared memory and dK, dV in TMEM for the whole loop over
-//          the query heads of the group and their query blocks (64 rows,
-//          two blocks' scores in TMEM at once), so dK and dV need no
-//          atomics.  Per step (key rows on the 128 TMEM lanes):
+//          the query heads of the group and their query blocks, so dK and dV
+//          need no atomics.  Per step (key rows on the 128 TMEM lanes):
 //              S^T = (K-c) Q_i^T      dP^T = V dO_i^T       (tcgen05, SMEM x SMEM)
 //              P^T = exp2(S^T * scale*log2e - L2_i),  dS^T = P^T * (dP^T - D_i)
-//                                                           (one thread per key row
-//                                                            and 32 query columns)
+//                                                           (one thread per key row)
 //              dV += P^T dO_i         dK += dS^T Q_i        (tcgen05, A from TMEM)
 //              dQ_i^T = (K-c)^T dS^T                        (tcgen05, SMEM x SMEM)
-//          and a readout warpgroup adds dQ_i^T into the f32 accumulator with
-//          float32 reductions.  MMA order per step: dV, dK, dQ^T (i), then
-//          S^T (i+1), then -- once dQ^T (i) is in registers -- dP^T (i+1),
-//          which takes dQ^T's TMEM columns.  Q_i, dO_i and the row vectors
-//          L2_i, D_i arrive through a ring of TMA copies;
+//          and readout warps add dQ_i^T into the f32 accumulator with float32
+//          reductions.  Q_i, dO_i and the row vectors L2_i, D_i arrive
+//          through a ring of TMA copies.
+//          d = 64, 128: bwd_wide_kernel, 128-row query blocks, one TMEM score
+//          set and a two-phase elementwise stage (see its comment block).
+//          d = 256: the dK and dV accumulators alone fill TMEM, so
+//          bwd_kernel runs two passes over the same key blocks, dV (S^T,
+//          P^T, dV) then dK and dQ, with 64-row query blocks and two TMEM
+//          score sets so one block's elementwise work overlaps the next
+//          block's MMAs;
 //   dq     dQ = bf16(scale * accumulator).
-// For d = 256 the dK and dV accumulators alone fill TMEM, so dkdv runs two
-// passes over the same key blocks: dV (S^T, P^T, dV), then dK and dQ.
 #include <math.h>
 
 #include <type_traits>
@@ -51,11 +52,13 @@
 namespace fa {
 namespace {
 
-// Warp roles: 0-7 elementwise stage (two warpgroups, half of the query
-// columns each, 32 at a time; each also reads out and reduces a quarter of
-// dQ^T), 8-11 dQ readout (the other half of dQ^T), 12 TMA producer, 13 MMA
-// issuer.  The producer and MMA roles run in lane 0 alone (measured ~8%
-// faster on B200 than keeping the warp converged around each wait).
+// bwd_kernel warp roles: 0-7 elementwise stage (two warpgroups, half of the
+// query columns each, 32 at a time; each also reads out and reduces a quarter
+// of dQ^T when a step has four 32-column chunks), 8-11 dQ readout, 12 TMA
+// producer, 13 MMA issuer.  The producer and MMA roles run in lane 0 alone
+// (measured ~8% faster on B200 than keeping the warp converged around each
+// wait).  Its single-pass mode (kFull) serves d <= 128 when selected; the
+// library launches bwd_wide_kernel there instead.
 constexpr int kThreads = 448;
 constexpr int kReadoutWarp0 = 8;
 constexpr int kProducerWarp = 12;
