@@ -32,6 +32,11 @@
 // causal mask may be bottom-right aligned there (key j hidden from query i
 // when j > i + Nk - Nq).
 //
+// Dropout (DROP instances): P written to TMEM keeps only the elements whose
+// Philox4x32-10 word is >= floor(p 2^32) (one counter per four key columns of
+// a row); the row sum uses the undropped P and the epilogue scales O by
+// 1 / (1 - p).
+//
 // MMA issue order per block j (two tiles): PV0(j), S0(j+1), PV1(j), S1(j+1):
 // the softmax of one tile overlaps the tensor-core work of the other.
 // tcgen05 ops of one thread complete in issue order, and tcgen05.commit
