@@ -516,7 +516,23 @@ int run_fwd(const AttnArgs &a) {
 }
 
 // Merge the pieces of a split-KV forward, one warp per query row:
-// L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s -> bf16.
+// L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s -> bf16.  The pieces'
+// log-sum-exps are reduced across the lanes first; the weighted sum then
+// keeps four pieces' loads in flight at a time.
+template <int PER>
+__device__ __forceinline__ void load_row_slice(const float *src, float (&v)[PER]) {
+  if constexpr (PER == 2) {
+    const float2 t = *reinterpret_cast<const float2 *>(src);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+#pragma unroll
+    for (int e = 0; e < PER; e += 4) {
+      const float4 t = *reinterpret_cast<const float4 *>(src + e);
+      v[e] = t.x; v[e + 1] = t.y; v[e + 2] = t.z; v[e + 3] = t.w;
+    }
+  }
+}
+
 template <int D>
 __global__ void splitkv_combine_kernel(const float *__restrict__ o_part,
                                        const float *__restrict__ l_part, __nv_bfloat16 *__restrict__ o,
@@ -524,22 +540,48 @@ __global__ void splitkv_combine_kernel(const float *__restrict__ o_part,
   const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
+  const float *lp = l_part + row;
   float m = -INFINITY;
-  for (int s = 0; s < splits; ++s) m = fmaxf(m, l_part[(size_t)s * rows + row]);
+  for (int s = lane; s < splits; s += 32) m = fmaxf(m, lp[(size_t)s * rows]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float tot = 0.f;
+  if (m != -INFINITY) {
+    for (int s = lane; s < splits; s += 32) {
+      const float ls = lp[(size_t)s * rows];
+      tot += ls == -INFINITY ? 0.f : __expf(ls - m);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
+  }
   constexpr int PER = D / 32;   // 2, 4 or 8 elements per lane
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  float tot = 0.f;
-  if (m != -INFINITY) {
-    for (int s = 0; s < splits; ++s) {
-      const float ls = l_part[(size_t)s * rows + row];
-      if (ls == -INFINITY) continue;
-      const float w = __expf(ls - m);
-      tot += w;
-      const float *src = o_part + ((size_t)s * rows + row) * D + lane * PER;
+  if (tot > 0.f) {
+    const float *op = o_part + row * D + lane * PER;
+    const size_t piece = (size_t)rows * D;
+    int s = 0;
+    for (; s + 4 <= splits; s += 4) {
+      float w[4], v[4][PER];
 #pragma unroll
-      for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+      for (int u = 0; u < 4; ++u) {
+        const float ls = lp[(size_t)(s + u) * rows];
+        w[u] = ls == -INFINITY ? 0.f : __expf(ls - m);
+        load_row_slice<PER>(op + (size_t)(s + u) * piece, v[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = fmaf(w[u], v[u][e], acc[e]);
+    }
+    for (; s < splits; ++s) {
+      const float ls = lp[(size_t)s * rows];
+      const float w = ls == -INFINITY ? 0.f : __expf(ls - m);
+      float v[PER];
+      load_row_slice<PER>(op + (size_t)s * piece, v);
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, v[e], acc[e]);
     }
   }
   const float inv = tot > 0.f ? 1.f / tot : 0.f;
