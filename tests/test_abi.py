@@ -153,3 +153,13 @@ def test_dropout_argument_errors():
     assert fwd(0.1, d=96) == F.FA_ERR_UNSUPPORTED
     assert bwd(0.1, d=256) == F.FA_ERR_UNSUPPORTED      # dropout backward: d = 64, 128
     assert fwd(0.1, ptrs=(FAKE + 2,) + (FAKE,) * 4) == F.FA_ERR_ALIGNMENT
+
+
+def test_size_limits():
+    """Sizes past the kernels' index arithmetic are refused before any launch."""
+    f = F.fa_fwd
+    big_n = (1 << 28) + 1
+    assert f(*(FAKE,) * 5, 1, 1, 1, big_n, 8, 64, 0.125, 0) == F.FA_ERR_UNSUPPORTED
+    assert f(*(FAKE,) * 5, 1, 1, 1, 8, big_n, 64, 0.125, 0) == F.FA_ERR_UNSUPPORTED
+    # B*Hq*Nq*d above 4e12 elements
+    assert f(*(FAKE,) * 5, 4096, 1024, 1024, 8192, 8, 128, 0.125, 0) == F.FA_ERR_UNSUPPORTED
