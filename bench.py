@@ -72,10 +72,11 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix=f"fa_clocks_rank{index}_", suffix=".csv")
+        os.close(fd)
 
     def start(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
         cmd = ["nvidia-smi", f"--id={self.index}",
                "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -89,6 +90,10 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         try:
@@ -111,6 +116,10 @@ class ClockSampler:
                 for nm, val in zip(names, parts[5:9]):
                     if val.lower() == "active":
                         reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not sms:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
