@@ -51,7 +51,7 @@ typedef struct CUstream_st *fa_stream_t;
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null pointer, size <= 0, Hq % Hkv != 0, scale not finite or <= 0 */
-  FA_ERR_UNSUPPORTED = 2, /* head dim or mask combination this build does not run */
+  FA_ERR_UNSUPPORTED = 2, /* head dim, length or mask combination the library does not run */
   FA_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
   FA_ERR_ARCH = 4,        /* current device is not compute capability 10.0 */
   FA_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
@@ -197,7 +197,7 @@ int fa_bwd_f32(const float *q, const float *k, const float *v, const float *o,
  * synchronisation cudaMalloc can cause).  Same arguments and results as
  * fa_bwd, minus the workspace: the scratch lives in one fixed 32 MiB array
  * inside the library (reserved on every GPU that loads it, until exit).
- * The pages have no counterpart; this is an interface convenience.
+ * The FlashAttention pages describe no such call; it is an interface convenience.
  * Returns FA_ERR_UNSUPPORTED, without touching the device, when the problem
  * needs more scratch than that (about 4*B*Hq*(Nq*(d+2) + d) bytes plus
  * padding, e.g. more than about 64,000 query rows B*Hq*Nq at d = 128).  The first call on a

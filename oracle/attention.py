@@ -17,9 +17,9 @@ What it computes (the plain definition, materialised, in float64):
 * Saved statistic -- the blog's section 2.3 keeps m and l per row; this oracle
   returns the single per-row log-sum-exp L = m + ln(l) of the scaled scores,
   natural log.
-* Backward -- the pages only say that P is recomputed from Q, K and the saved
-  statistics (blog section 2.3).  The gradients below are the calculus of the
-  forward definition for the scalar f = sum(O * dO):
+* Backward -- the FlashAttention blog (section 2.3) only says that P is
+  recomputed from Q, K and the saved statistics.  The gradients below are the
+  calculus of the forward definition for the scalar f = sum(O * dO):
       dV = P^T dO,  dP = dO V^T,  D_i = sum_j P_ij dP_ij (= sum_d dO_id O_id),
       dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q.
   Pinned by central finite differences and a library cross-check in tests.
@@ -27,9 +27,10 @@ What it computes (the plain definition, materialised, in float64):
   query head h reads key/value head floor(h / g), g = Hq / Hkv; dK and dV of a
   key/value head sum over the g query heads of its group.
 * Causal alignment when Nq < Nk (inference: the Nq queries are the last Nq
-  positions of a sequence whose Nk keys are all cached) -- the pages only use
-  Nq = Nk.  Reading adopted: bottom-right alignment, key j is masked for
-  query i when j > i + (Nk - Nq); it equals the top-left mask when Nq = Nk.
+  positions of a sequence whose Nk keys are all cached) -- the blog and the
+  CSDN tutorial only use Nq = Nk.  Reading adopted: bottom-right alignment,
+  key j is masked for query i when j > i + (Nk - Nq); it equals the top-left
+  mask when Nq = Nk.
   Selected with ``causal_offset = Nk - Nq``; the default 0 is top-left.
 * Split-KV forward and the merge of partial results -- the key range of a
   row is cut into pieces, each piece gives (O_s, L_s) over its own keys, and
@@ -38,7 +39,7 @@ What it computes (the plain definition, materialised, in float64):
       L = log sum_s exp(L_s),   O = sum_s exp(L_s - L) O_s.
   A piece that sees no key of a row has L_s = -inf and contributes nothing.
 * Dropout on P (the blog's section 5 call passes dropout_p to
-  F.scaled_dot_product_attention; the pages use 0).  Reading adopted: inverted
+  F.scaled_dot_product_attention with 0).  Reading adopted: inverted
   dropout of the normalised probabilities, O = (P * Z) V / (1 - p) with
   Z_ij in {0, 1}, while L stays the log-sum-exp of the undropped scores.  The
   mask is a pure function of (seed, offset, batch*Hq + head, i, j): the

@@ -1,5 +1,5 @@
 """Pins for the float64 oracle: closed forms, invariants, finite differences,
-a library cross-check and the pages' own worked setup.  CPU only.
+a library cross-check and the CSDN tutorial's own worked setup.  CPU only.
 
 Each check is written as a function of an oracle "implementation" so the same
 checks can be run against planted mistakes (``test_pins_catch_mutants``): a
@@ -309,7 +309,7 @@ def test_oracle_pin(pin):
 
 
 # ---------------------------------------------------------------------------
-# the block-wise recurrences of the pages equal the one-shot softmax
+# the block-wise recurrences (blog section 2.2 and 4.1) equal the one-shot softmax
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("causal", [False, True])
