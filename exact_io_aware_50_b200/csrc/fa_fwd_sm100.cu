@@ -16,6 +16,13 @@
 // same quantity (the wiki's FlashAttention-4 paragraph lists conditional
 // rescaling; the exactness argument is the deferred-normalisation identity).
 //
+// Persistent CTAs (one per SM): each runs a fixed sequence of work units,
+// keeping its TMEM, barriers and rings; the next unit's Q load and first S
+// MMAs overlap the previous unit's epilogue.  Q is refilled once the last S
+// of a unit has read it (barrier q_empty), O once the epilogue has read it
+// out (o_empty).  Barrier phases follow running counters of key blocks and
+// units across the sequence.
+//
 // Warp roles (10 warps, 320 threads, one CTA per SM):
 //   warps 0-3  softmax + epilogue for Q tile 0 (thread = TMEM lane = row)
 //   warps 4-7  softmax + epilogue for Q tile 1 (NT == 2)
@@ -76,8 +83,8 @@ struct FwdCfg {
   static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NT],
-  // p_full[NT], o_full[NT], drain
-  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NT + 1;
+  // p_full[NT], o_full[NT], drain, q_empty, o_empty[NT]
+  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NT + 1 + 1 + NT;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem base slot, abort flag
   static constexpr int SMEM = OFF_MISC + 16 + 1024;       // + alignment slack
   // TMEM columns
@@ -122,47 +129,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             B_VEMPTY = 1 + 3 * C::STAGES;
   const int B_SFULL = 1 + 4 * C::STAGES, B_PFULL = B_SFULL + C::NT, B_OFULL = B_PFULL + C::NT;
   const int B_DRAIN = B_OFULL + C::NT;
+  const int B_QEMPTY = B_DRAIN + 1, B_OEMPTY = B_DRAIN + 2;
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
 
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
 
-  // Work unit.  Causal: the heaviest query blocks of every head first, so the
-  // last wave holds the shortest units.  Otherwise all units cost the same and
-  // they run head by head, so the K and V tiles a wave reads are those of a
-  // few heads and stay in L2.
-  // Split-KV: the piece index is the slowest-varying part of the unit.
+  // Persistent CTAs: round k gives CTA c unit k*G + c (k even) or
+  // k*G + G-1-c (k odd), G = gridDim.x.  Unit order:
+  // causal, the heaviest query blocks of every head first; otherwise head by
+  // head, so the K and V tiles a wave reads are those of a few heads and stay
+  // in L2.  Split-KV: the piece index is the slowest-varying part.
   const int per_piece = p.nqb * p.BH;
-  const int piece = blockIdx.x / per_piece;
-  const int unit = blockIdx.x % per_piece;
-  const int qblk = p.causal ? p.nqb - 1 - unit / p.BH : unit % p.nqb;
-  const int bh = p.causal ? unit % p.BH : unit / p.nqb;
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int bh_kv = b * p.Hkv + h / (p.Hq / p.Hkv);
-  const int q_start = qblk * C::NT * BM;
-  const int nkb_all = (p.Nk + C::BN - 1) / C::BN;
-  const int nkb_vis =
-      p.causal ? min(nkb_all, (q_start + C::NT * BM + p.causal_off + C::BN - 1) / C::BN) : nkb_all;
-  // key blocks [j0, j0 + nkb) of this piece
-  const int per_split = (nkb_vis + p.splits - 1) / p.splits;
-  const int j0 = min(nkb_vis, piece * per_split);
-  const int nkb = min(nkb_vis, j0 + per_split) - j0;
-  if (nkb == 0) {
-    // An empty piece (only in split mode): its rows see no key here.
-    for (int i = threadIdx.x; i < C::NT * BM; i += blockDim.x) {
-      const int row = q_start + i;
-      if (row >= p.Nq) break;
-      const size_t prow = ((size_t)piece * p.BH + bh) * p.Nq + row;
-      p.l_part[prow] = -INFINITY;
-      float4 *orow = reinterpret_cast<float4 *>(p.o_part + prow * C::D);
-      for (int e = 0; e < C::D / 4; ++e) orow[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    return;
-  }
+  const int total_units = per_piece * p.splits;
+  struct Unit {
+    int piece, bh, bh_kv, q_start, j0, nkb;
+  };
+  auto decode = [&](int u) {
+    Unit U;
+    U.piece = u / per_piece;
+    const int v = u % per_piece;
+    const int qblk = p.causal ? p.nqb - 1 - v / p.BH : v % p.nqb;
+    U.bh = p.causal ? v % p.BH : v / p.nqb;
+    const int b = U.bh / p.Hq, h = U.bh % p.Hq;
+    U.bh_kv = b * p.Hkv + h / (p.Hq / p.Hkv);
+    U.q_start = qblk * C::NT * BM;
+    const int nkb_all = (p.Nk + C::BN - 1) / C::BN;
+    const int nkb_vis = p.causal
+                            ? min(nkb_all, (U.q_start + C::NT * BM + p.causal_off + C::BN - 1) / C::BN)
+                            : nkb_all;
+    // key blocks [j0, j0 + nkb) of this piece
+    const int per_split = (nkb_vis + p.splits - 1) / p.splits;
+    U.j0 = min(nkb_vis, U.piece * per_split);
+    U.nkb = min(nkb_vis, U.j0 + per_split) - U.j0;
+    return U;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
+    mbar_init(bar(B_QEMPTY), 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
       mbar_init(bar(B_KEMPTY + s), 1);
@@ -173,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_SFULL + t), 1);
       mbar_init(bar(B_PFULL + t), BM);
       mbar_init(bar(B_OFULL + t), 1);
+      mbar_init(bar(B_OEMPTY + t), BM);
     }
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -193,39 +200,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   WaitCtx wc{p.err, abort_flag, kWaitLimitNs};
 
+  // Ring positions run on across units: g counts key blocks, uq units with
+  // work (barrier phases are these counters' parities).
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     // The whole role runs in lane 0; the other lanes wait at the end.
     if (lane == 0) {
       int last_k_phase[C::STAGES], last_v_phase[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) last_k_phase[s] = last_v_phase[s] = -1;
+      int last_q_phase = -1;
       bool ok = true;
-      mbar_arrive_expect_tx(bar(B_QFULL), C::NT * C::Q_TILE);
-      for (int t = 0; t < C::NT; ++t)
-        for (int c = 0; c < C::DCH; ++c)
-          tma_load_3d(sbase + C::OFF_Q + t * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(B_QFULL),
-                      c * 64, q_start + t * BM, bh);
-      for (int j = 0; j < nkb && ok; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        ok = bounded_wait(bar(B_KEMPTY + s), ph ^ 1, wc);
+      int g = 0, uq = 0;
+      for (int k = 0; ok && k * (int)gridDim.x < total_units; ++k) {
+        // snake order: even rounds ascending, odd rounds descending, so the
+        // heavy-first unit list pairs heavy with light units on each CTA
+        const int u = k * (int)gridDim.x +
+                      ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+        if (u >= total_units) continue;
+        const Unit U = decode(u);
+        if (U.nkb == 0) continue;
+        // the previous unit's S MMAs must be done with the Q tiles
+        ok = bounded_wait(bar(B_QEMPTY), (uq & 1) ^ 1, wc);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(B_KFULL + s), C::KV_TILE);
-        for (int c = 0; c < C::DCH; ++c)
-          tma_load_3d(sbase + C::OFF_K + s * C::KV_TILE + c * C::KV_CHUNK, &tmK, bar(B_KFULL + s),
-                      c * 64, (j0 + j) * C::BN, bh_kv);
-        last_k_phase[s] = ph;
-        ok = bounded_wait(bar(B_VEMPTY + s), ph ^ 1, wc);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar(B_VFULL + s), C::KV_TILE);
-        for (int c = 0; c < C::DCH; ++c)
-          tma_load_3d(sbase + C::OFF_V + s * C::KV_TILE + c * C::KV_CHUNK, &tmV, bar(B_VFULL + s),
-                      c * 64, (j0 + j) * C::BN, bh_kv);
-        last_v_phase[s] = ph;
+        mbar_arrive_expect_tx(bar(B_QFULL), C::NT * C::Q_TILE);
+        for (int t = 0; t < C::NT; ++t)
+          for (int c = 0; c < C::DCH; ++c)
+            tma_load_3d(sbase + C::OFF_Q + t * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(B_QFULL),
+                        c * 64, U.q_start + t * BM, U.bh);
+        last_q_phase = uq & 1;
+        for (int j = 0; j < U.nkb && ok; ++j, ++g) {
+          const int s = g % C::STAGES;
+          const uint32_t ph = (g / C::STAGES) & 1;
+          ok = bounded_wait(bar(B_KEMPTY + s), ph ^ 1, wc);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(B_KFULL + s), C::KV_TILE);
+          for (int c = 0; c < C::DCH; ++c)
+            tma_load_3d(sbase + C::OFF_K + s * C::KV_TILE + c * C::KV_CHUNK, &tmK,
+                        bar(B_KFULL + s), c * 64, (U.j0 + j) * C::BN, U.bh_kv);
+          last_k_phase[s] = ph;
+          ok = bounded_wait(bar(B_VEMPTY + s), ph ^ 1, wc);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(B_VFULL + s), C::KV_TILE);
+          for (int c = 0; c < C::DCH; ++c)
+            tma_load_3d(sbase + C::OFF_V + s * C::KV_TILE + c * C::KV_CHUNK, &tmV,
+                        bar(B_VFULL + s), c * 64, (U.j0 + j) * C::BN, U.bh_kv);
+          last_v_phase[s] = ph;
+        }
+        ++uq;
       }
       if (!ok) {
         // Drain: let every copy this role issued land before the CTA exits.
-        (void)drain_wait(bar(B_QFULL), 0, p.err, kWaitLimitNs);
+        if (last_q_phase >= 0) (void)drain_wait(bar(B_QFULL), last_q_phase, p.err, kWaitLimitNs);
         for (int s = 0; s < C::STAGES; ++s) {
           if (last_k_phase[s] >= 0) (void)drain_wait(bar(B_KFULL + s), last_k_phase[s], p.err, kWaitLimitNs);
           if (last_v_phase[s] >= 0) (void)drain_wait(bar(B_VFULL + s), last_v_phase[s], p.err, kWaitLimitNs);
@@ -263,41 +288,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // The whole role runs in lane 0; the other lanes wait at the end.
     if (lane == 0) {
-      bool ok = bounded_wait(bar(B_QFULL), 0, wc);
-      if (ok) ok = bounded_wait(bar(B_KFULL + 0), 0, wc);
-      if (ok) {
+      bool ok = true;
+      int g = 0, uq = 0;
+      for (int k = 0; ok && k * (int)gridDim.x < total_units; ++k) {
+        // snake order: even rounds ascending, odd rounds descending, so the
+        // heavy-first unit list pairs heavy with light units on each CTA
+        const int u = k * (int)gridDim.x +
+                      ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+        if (u >= total_units) continue;
+        const Unit U = decode(u);
+        if (U.nkb == 0) continue;
+        ok = bounded_wait(bar(B_QFULL), uq & 1, wc);
+        if (ok) ok = bounded_wait(bar(B_KFULL + g % C::STAGES), (g / C::STAGES) & 1, wc);
+        if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < C::NT; ++t) {
-          issue_S(t, 0);
+          issue_S(t, g % C::STAGES);
           mma_commit(bar(B_SFULL + t));
         }
-        mma_commit(bar(B_KEMPTY + 0));
-      }
-      for (int j = 0; j < nkb && ok; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        const int s1 = (j + 1) % C::STAGES;
-        const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-        ok = bounded_wait(bar(B_VFULL + s), ph, wc);
-        if (!ok) break;
-        for (int t = 0; t < C::NT && ok; ++t) {
-          ok = bounded_wait(bar(B_PFULL + t), j & 1, wc);
+        mma_commit(bar(B_KEMPTY + g % C::STAGES));
+        if (U.nkb == 1) mma_commit(bar(B_QEMPTY));   // last S of the unit issued
+        for (int j = 0; j < U.nkb && ok; ++j) {
+          const int gj = g + j;
+          const int s = gj % C::STAGES;
+          const uint32_t ph = (gj / C::STAGES) & 1;
+          const int s1 = (gj + 1) % C::STAGES;
+          const uint32_t ph1 = ((gj + 1) / C::STAGES) & 1;
+          ok = bounded_wait(bar(B_VFULL + s), ph, wc);
           if (!ok) break;
-          if (t == 0 && j + 1 < nkb) {
-            ok = bounded_wait(bar(B_KFULL + s1), ph1, wc);
+          for (int t = 0; t < C::NT && ok; ++t) {
+            ok = bounded_wait(bar(B_PFULL + t), gj & 1, wc);
             if (!ok) break;
+            if (t == 0 && j + 1 < U.nkb) {
+              ok = bounded_wait(bar(B_KFULL + s1), ph1, wc);
+              if (!ok) break;
+            }
+            if (j == 0 && uq > 0) {
+              // the previous unit's epilogue must have read O_t out of TMEM
+              ok = bounded_wait(bar(B_OEMPTY + t), (uq - 1) & 1, wc);
+              if (!ok) break;
+            }
+            tc_fence_after();
+            issue_PV(t, s, j == 0);
+            if (j + 1 < U.nkb) {
+              issue_S(t, s1);
+              mma_commit(bar(B_SFULL + t));
+              if (t == C::NT - 1) {
+                mma_commit(bar(B_KEMPTY + s1));
+                if (j + 2 == U.nkb) mma_commit(bar(B_QEMPTY));   // last S of the unit
+              }
+            } else {
+              mma_commit(bar(B_OFULL + t));
+            }
+            if (t == C::NT - 1) mma_commit(bar(B_VEMPTY + s));
           }
-          tc_fence_after();
-          issue_PV(t, s, j == 0);
-          if (j + 1 < nkb) {
-            issue_S(t, s1);
-            mma_commit(bar(B_SFULL + t));
-            if (t == C::NT - 1) mma_commit(bar(B_KEMPTY + s1));
-          } else {
-            mma_commit(bar(B_OFULL + t));
-          }
-          if (t == C::NT - 1) mma_commit(bar(B_VEMPTY + s));
         }
+        g += U.nkb;
+        ++uq;
       }
       if (!ok) {
         // Drain: every MMA issued so far must finish before TMEM is freed.
@@ -310,150 +357,176 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;                  // Q tile of this warpgroup
     const int r = threadIdx.x & 127;          // row within the tile = TMEM lane
-    const int row = q_start + t * BM + r;     // query row
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::TM_S + t * C::BN;
     const uint32_t tP = tS + C::BN / 2;
     const uint32_t tO = tmem + lane_off + C::TM_O + t * C::D;
-    const int row_lo = q_start + t * BM;
-    // keys [0, limit) visible
-    const int limit_row = p.causal ? min(p.Nk, row + 1 + p.causal_off) : p.Nk;
-    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkb; ++j) {
-      ok = warp_wait_all(bar(B_SFULL + t), j & 1, wc);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[C::BN];
-#pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c)
-        tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-      tmem_wait_ld();
-      float *s = reinterpret_cast<float *>(sr);
-      const int col_lo = (j0 + j) * C::BN;
-      const bool need_mask =
-          (col_lo + C::BN > p.Nk) || (p.causal && col_lo + C::BN - 1 > row_lo + p.causal_off);
-      if (need_mask) {
-        const int lim = limit_row - col_lo;
-#pragma unroll
-        for (int c = 0; c < C::BN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+    int g = 0, uq = 0;
+    for (int k = 0; ok && k * (int)gridDim.x < total_units; ++k) {
+        // snake order: even rounds ascending, odd rounds descending, so the
+        // heavy-first unit list pairs heavy with light units on each CTA
+        const int u = k * (int)gridDim.x +
+                      ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+        if (u >= total_units) continue;
+      const Unit U = decode(u);
+      const int bh = U.bh;
+      const int row = U.q_start + t * BM + r;     // query row
+      if (U.nkb == 0) {
+        // An empty piece (only in split mode): its rows see no key here.
+        if (row < p.Nq) {
+          const size_t prow = ((size_t)U.piece * p.BH + bh) * p.Nq + row;
+          p.l_part[prow] = -INFINITY;
+          float4 *orow = reinterpret_cast<float4 *>(p.o_part + prow * C::D);
+          for (int e = 0; e < C::D / 4; ++e) orow[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        continue;
       }
-      // row max: eight independent partial maxima, then a small tree
-      float mp[8];
+      const int row_lo = U.q_start + t * BM;
+      // keys [0, limit) visible
+      const int limit_row = p.causal ? min(p.Nk, row + 1 + p.causal_off) : p.Nk;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < U.nkb; ++j) {
+        ok = warp_wait_all(bar(B_SFULL + t), (g + j) & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[C::BN];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mp[u] = s[u];
-#pragma unroll
-      for (int c = 8; c < C::BN; c += 8)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mp[u] = fmaxf(mp[u], s[c + u]);
-      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      const float m_new = fmaxf(m_run, mx * p.scale_log2);
-      bool rescale = false;
-      float alpha = 1.f;
-      if (j == 0) {
-        m_run = m_new;
-      } else if (__any_sync(0xffffffffu, m_new - m_run > kRescaleThreshold)) {
-        rescale = true;
-        alpha = fast_exp2(m_run - m_new);
-        m_run = m_new;
-      }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // p = 2^(s * scale * log2e - m) on MUFU (exp2_poly for one column in
-      // four when FA_FWD_POLY_EXP is set); row sum in four independent
-      // partials over the undropped p; with dropout, P in TMEM keeps only the
-      // columns whose Philox word is >= drop_thr (one Philox call per four
-      // key columns)
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c) {
-        uint32_t pk[16];
-        uint4 rnd = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float x0 = fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_use);
-          const float x1 = fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_use);
-          const float p0 = fast_exp2(x0);
-          const float p1 = (kPolyExp && (e & 1)) ? exp2_poly(x1) : fast_exp2(x1);
-          rs[e & 3] += p0 + p1;
-          if (DROP) {
-            if ((e & 1) == 0)
-              rnd = philox4x32_10((uint32_t)(col_lo + c * 32 + 2 * e) >> 2, (uint32_t)row,
-                                  (uint32_t)bh, p.drop_off, p.seed_lo, p.seed_hi);
-            const uint32_t w0 = (e & 1) ? rnd.z : rnd.x, w1 = (e & 1) ? rnd.w : rnd.y;
-            pk[e] = pack_bf16x2(w0 >= p.drop_thr ? p0 : 0.f, w1 >= p.drop_thr ? p1 : 0.f);
-          } else {
-            pk[e] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < C::BN / 32; ++c)
+          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_wait_ld();
+        float *s = reinterpret_cast<float *>(sr);
+        const int col_lo = (U.j0 + j) * C::BN;
+        const bool need_mask =
+            (col_lo + C::BN > p.Nk) || (p.causal && col_lo + C::BN - 1 > row_lo + p.causal_off);
+        if (need_mask) {
+          const int lim = limit_row - col_lo;
+  #pragma unroll
+          for (int c = 0; c < C::BN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+        }
+        // row max: eight independent partial maxima, then a small tree
+        float mp[8];
+  #pragma unroll
+        for (int u = 0; u < 8; ++u) mp[u] = s[u];
+  #pragma unroll
+        for (int c = 8; c < C::BN; c += 8)
+  #pragma unroll
+          for (int u = 0; u < 8; ++u) mp[u] = fmaxf(mp[u], s[c + u]);
+        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        const float m_new = fmaxf(m_run, mx * p.scale_log2);
+        bool rescale = false;
+        float alpha = 1.f;
+        if (j == 0) {
+          m_run = m_new;
+        } else if (__any_sync(0xffffffffu, m_new - m_run > kRescaleThreshold)) {
+          rescale = true;
+          alpha = fast_exp2(m_run - m_new);
+          m_run = m_new;
+        }
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        // p = 2^(s * scale * log2e - m) on MUFU (exp2_poly for one column in
+        // four when FA_FWD_POLY_EXP is set); row sum in four independent
+        // partials over the undropped p; with dropout, P in TMEM keeps only the
+        // columns whose Philox word is >= drop_thr (one Philox call per four
+        // key columns)
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll
+        for (int c = 0; c < C::BN / 32; ++c) {
+          uint32_t pk[16];
+          uint4 rnd = make_uint4(0, 0, 0, 0);
+  #pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_use);
+            const float x1 = fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_use);
+            const float p0 = fast_exp2(x0);
+            const float p1 = (kPolyExp && (e & 1)) ? exp2_poly(x1) : fast_exp2(x1);
+            rs[e & 3] += p0 + p1;
+            if (DROP) {
+              if ((e & 1) == 0)
+                rnd = philox4x32_10((uint32_t)(col_lo + c * 32 + 2 * e) >> 2, (uint32_t)row,
+                                    (uint32_t)bh, p.drop_off, p.seed_lo, p.seed_hi);
+              const uint32_t w0 = (e & 1) ? rnd.z : rnd.x, w1 = (e & 1) ? rnd.w : rnd.y;
+              pk[e] = pack_bf16x2(w0 >= p.drop_thr ? p0 : 0.f, w1 >= p.drop_thr ? p1 : 0.f);
+            } else {
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+          }
+          tmem_st16(tP + c * 16, pk);
+        }
+        const float rowsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        l_run = l_run * alpha + rowsum;
+        if (rescale) {
+  #pragma unroll 1
+          for (int c = 0; c < C::D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c * 32, ov);
+            tmem_wait_ld();
+  #pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tO + c * 32, ov);
           }
         }
-        tmem_st16(tP + c * 16, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + t));
       }
-      const float rowsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      l_run = l_run * alpha + rowsum;
-      if (rescale) {
-#pragma unroll 1
+      // ---------------------------------------------------------- epilogue
+      if (ok) ok = warp_wait_all(bar(B_OFULL + t), uq & 1, wc);
+      if (ok && p.splits > 1) {
+        // normalised partial output and log-sum-exp of this piece; a row whose
+        // keys in the piece are all hidden has l = 0: O_s = 0, L_s = -inf
+        tc_fence_after();
+        const bool empty = !(l_run > 0.f);
+        const float inv_l = empty ? 0.f : 1.f / l_run;
+        const bool live = row < p.Nq;
+        const size_t prow = ((size_t)U.piece * p.BH + bh) * p.Nq + (live ? row : 0);
+        float4 *orow = reinterpret_cast<float4 *>(p.o_part + prow * C::D);
+  #pragma unroll 1
         for (int c = 0; c < C::D / 32; ++c) {
           uint32_t ov[32];
           tmem_ld32(tO + c * 32, ov);
           tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(tO + c * 32, ov);
+          if (live) {
+  #pragma unroll
+            for (int e = 0; e < 8; ++e)
+              orow[c * 8 + e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
+                                            __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                            __uint_as_float(ov[4 * e + 2]) * inv_l,
+                                            __uint_as_float(ov[4 * e + 3]) * inv_l);
+          }
         }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_PFULL + t));
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok) ok = warp_wait_all(bar(B_OFULL + t), 0, wc);
-    if (ok && p.splits > 1) {
-      // normalised partial output and log-sum-exp of this piece; a row whose
-      // keys in the piece are all hidden has l = 0: O_s = 0, L_s = -inf
-      tc_fence_after();
-      const bool empty = !(l_run > 0.f);
-      const float inv_l = empty ? 0.f : 1.f / l_run;
-      const bool live = row < p.Nq;
-      const size_t prow = ((size_t)piece * p.BH + bh) * p.Nq + (live ? row : 0);
-      float4 *orow = reinterpret_cast<float4 *>(p.o_part + prow * C::D);
-#pragma unroll 1
-      for (int c = 0; c < C::D / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(tO + c * 32, ov);
-        tmem_wait_ld();
-        if (live) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            orow[c * 8 + e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
-                                          __uint_as_float(ov[4 * e + 1]) * inv_l,
-                                          __uint_as_float(ov[4 * e + 2]) * inv_l,
-                                          __uint_as_float(ov[4 * e + 3]) * inv_l);
+        tc_fence_before();
+        mbar_arrive(bar(B_OEMPTY + t));   // O_t read out: the next unit may overwrite it
+        if (live) p.l_part[prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      } else if (ok) {
+        tc_fence_after();
+        const float inv_l = (DROP ? p.drop_scale : 1.f) / l_run;
+        const bool live = row < p.Nq;
+        __nv_bfloat16 *orow = p.o + ((size_t)bh * p.Nq + (live ? row : 0)) * C::D;
+  #pragma unroll 1
+        for (int c = 0; c < C::D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c * 32, ov);
+          tmem_wait_ld();
+          uint32_t pk[16];
+  #pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
+                                __uint_as_float(ov[2 * e + 1]) * inv_l);
+          if (live) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+  #pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
         }
+        tc_fence_before();
+        mbar_arrive(bar(B_OEMPTY + t));   // O_t read out: the next unit may overwrite it
+        if (live) p.o_lse[(size_t)bh * p.Nq + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       }
-      if (live) p.l_part[prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
-    } else if (ok) {
-      tc_fence_after();
-      const float inv_l = (DROP ? p.drop_scale : 1.f) / l_run;
-      const bool live = row < p.Nq;
-      __nv_bfloat16 *orow = p.o + ((size_t)bh * p.Nq + (live ? row : 0)) * C::D;
-#pragma unroll 1
-      for (int c = 0; c < C::D / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(tO + c * 32, ov);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
-                              __uint_as_float(ov[2 * e + 1]) * inv_l);
-        if (live) {
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-        }
-      }
-      if (live) p.o_lse[(size_t)bh * p.Nq + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      g += U.nkb;
+      ++uq;
     }
   }
 
@@ -511,7 +584,12 @@ int run_fwd(const AttnArgs &a) {
     return 5;
   const long long units = (long long)p.nqb * p.BH * p.splits;
   if (units > 2147483647LL) return 2;
-  kern<<<(unsigned)units, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, p);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 5;
+  const long long grid = units < sms ? units : sms;
+  kern<<<(unsigned)grid, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }
 
