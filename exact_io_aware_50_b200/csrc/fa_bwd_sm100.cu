@@ -1140,9 +1140,10 @@ __global__ void bwd_center_kernel(const __nv_bfloat16 *__restrict__ k, float *__
   cvec[(size_t)blockIdx.x * D + t] = rintf(acc / (float)nr);
 }
 
-// Per padded query row (one warp each): D = sum_d dO * O and
+// Per padded query row: D = sum_d dO * O and
 // L2 = log2e * L - scale * log2e * (q . c) (rows past Nq: D = 0, L2 = +inf);
-// zero the row of the dQ accumulator.
+// zero the row of the dQ accumulator.  D / 8 lanes per row, each reading 16
+// bytes of O, dO and Q (so a warp covers 32 * 8 / D rows).
 template <int D>
 __global__ void bwd_preprocess_kernel(const __nv_bfloat16 *__restrict__ q,
                                       const __nv_bfloat16 *__restrict__ o,
@@ -1152,47 +1153,53 @@ __global__ void bwd_preprocess_kernel(const __nv_bfloat16 *__restrict__ q,
                                       float *__restrict__ l2, float *__restrict__ dq_acc,
                                       long long prow_total, int Nq, int npad, int Hq, int g,
                                       float scale_log2) {
-  const long long prow = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  constexpr int LPR = D / 8;     // lanes per row
+  constexpr int RPW = 32 / LPR;  // rows per warp
   const int lane = threadIdx.x & 31;
-  if (prow >= prow_total) return;
-  const long long bh = prow / npad;
-  const int qi = (int)(prow - bh * npad);
-  if (qi >= Nq) {
-    if (lane == 0) {
-      dsum[prow] = 0.f;
-      l2[prow] = INFINITY;
-    }
-    return;
-  }
+  const int l = lane % LPR;
+  const long long prow = ((long long)blockIdx.x * 8 + (threadIdx.x >> 5)) * RPW + lane / LPR;
+  const bool valid = prow < prow_total;
+  const long long bh = valid ? prow / npad : 0;
+  const int qi = valid ? (int)(prow - bh * npad) : 0;
+  const bool live = valid && qi < Nq;
   const long long row = bh * Nq + qi;
-  const int b = (int)(bh / Hq), h = (int)(bh % Hq);
-  const float *cv = cvec + ((size_t)b * (Hq / g) + h / g) * D;
-  constexpr int PER = D / 32;  // elements per lane (2, 4 or 8)
   float sd = 0.f, sq = 0.f;
-  const __nv_bfloat16 *orow = o + row * D + lane * PER;
-  const __nv_bfloat16 *drow = dout + row * D + lane * PER;
-  const __nv_bfloat16 *qrow = q + row * D + lane * PER;
+  if (live) {
+    const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+    const float *cv = cvec + ((size_t)b * (Hq / g) + h / g) * D + l * 8;
+    const uint4 ov = *reinterpret_cast<const uint4 *>(o + row * D + l * 8);
+    const uint4 dv = *reinterpret_cast<const uint4 *>(dout + row * D + l * 8);
+    const uint4 qv = *reinterpret_cast<const uint4 *>(q + row * D + l * 8);
+    const float4 c0 = *reinterpret_cast<const float4 *>(cv);
+    const float4 c1 = *reinterpret_cast<const float4 *>(cv + 4);
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w},
+                   qw[4] = {qv.x, qv.y, qv.z, qv.w};
+    const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-  for (int e = 0; e < PER; e += 2) {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(orow + e));
-    const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(drow + e));
-    const float2 qq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(qrow + e));
-    sd = fmaf(a.x, c.x, sd);
-    sd = fmaf(a.y, c.y, sd);
-    sq = fmaf(qq.x, cv[lane * PER + e], sq);
-    sq = fmaf(qq.y, cv[lane * PER + e + 1], sq);
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow[e]));
+      const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&dw[e]));
+      const float2 qq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qw[e]));
+      sd = fmaf(a.x, c.x, sd);
+      sd = fmaf(a.y, c.y, sd);
+      sq = fmaf(qq.x, cc[2 * e], sq);
+      sq = fmaf(qq.y, cc[2 * e + 1], sq);
+    }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
+  for (int off = LPR / 2; off > 0; off >>= 1) {
     sd += __shfl_xor_sync(0xffffffffu, sd, off);
     sq += __shfl_xor_sync(0xffffffffu, sq, off);
   }
-  if (lane == 0) {
-    dsum[prow] = sd;
-    l2[prow] = lse[row] * kLog2e - scale_log2 * sq;
+  if (valid && l == 0) {
+    dsum[prow] = live ? sd : 0.f;
+    l2[prow] = live ? lse[row] * kLog2e - scale_log2 * sq : INFINITY;
   }
-  float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D);
-  for (int e = lane; e < D / 4; e += 32) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (live) {
+    float4 *z = reinterpret_cast<float4 *>(dq_acc + row * D + l * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 // dQ = bf16(scale * acc), 8 elements per thread.
@@ -1241,7 +1248,9 @@ int run_prep(const AttnArgs &a) {
   if (cudaGetLastError() != cudaSuccess) return 5;
   const int npad = (int)ws_npad(a.Nq);
   const long long prows = (long long)a.B * a.Hq * npad;
-  bwd_preprocess_kernel<D><<<(unsigned)((prows + 7) / 8), 256, 0, a.stream>>>(
+  constexpr int rows_per_block = 8 * (256 / D);   // 8 warps, 32 * 8 / D rows each
+  bwd_preprocess_kernel<D><<<(unsigned)((prows + rows_per_block - 1) / rows_per_block), 256, 0,
+                             a.stream>>>(
       (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.o_in, (const __nv_bfloat16 *)a.dout,
       a.lse, w.cvec, w.dsum, w.l2, w.dq_acc, prows, a.Nq, npad, a.Hq, a.Hq / a.Hkv,
       a.scale * kLog2e);
