@@ -25,7 +25,7 @@ class Workload:
     N: int
     d: int
     causal: bool
-    dtype: str = "bf16"          # "bf16" or "f32"
+    dtype: str = "bf16"          # "bf16", "f32" or "e4m3"
     seed: int = 0
     q_mul: float = 1.0           # Q pre-multiplied in float32 before the cast
     k_add: float = 0.0           # constant added to every K element before the cast
@@ -75,7 +75,12 @@ SWEEP = _c5()
 INFER_PREFILL = Workload("inference_b1_h8_nq512_nk16384_d128", 1, 8, 8, 16384, 128, True, "bf16", 6,
                          backward=False, n_q=512)
 
-ALL = [SINGLE_HEAD_F32, TWO_BATCH_F32, TWO_BATCH_BF16, CAUSAL_TRAIN, LONG_GQA] + SWEEP + [INFER_PREFILL]
+# FP8 forward: the training shape with E4M3 inputs (forward only).
+FP8_CAUSAL = Workload("fp8_causal_b4_h16_n4096_d128", 4, 16, 16, 4096, 128, True, "e4m3", 7,
+                      backward=False)
+
+ALL = [SINGLE_HEAD_F32, TWO_BATCH_F32, TWO_BATCH_BF16, CAUSAL_TRAIN, LONG_GQA] + SWEEP + [INFER_PREFILL,
+                                                                                        FP8_CAUSAL]
 BY_NAME = {w.name: w for w in ALL}
 
 
@@ -110,6 +115,34 @@ def draw(B, Hq, Hkv, Nq, Nk, d, seed, dtype=torch.bfloat16, q_mul=1.0, k_add=0.0
     if k_add != 0.0:
         k = k + k_add
     return {name: t.to(dtype).contiguous() for name, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+
+
+E4M3_MAX = 448.0
+
+
+def draw_fp8(B, Hq, Hkv, N, d, seed, q_mul=1.0):
+    """E4M3 inputs: the float32 normals of ``draw`` for Q, K, V, each tensor
+    divided by one factor (its largest magnitude / 448, rounded to float32),
+    clamped to +-448 and cast by torch to float8_e4m3fn (round to nearest
+    even).  Returns uint8 code tensors q, k, v and the factors descale_q,
+    descale_k, descale_v (Python floats, exact float32 values)."""
+    t = draw(B, Hq, Hkv, N, N, d, seed, torch.float32, q_mul)
+    out = {}
+    for name in ("q", "k", "v"):
+        x = t[name]
+        amax = float(x.abs().max())
+        ds = float(torch.tensor(max(amax, 1e-30) / E4M3_MAX, dtype=torch.float32))
+        codes = (x / ds).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn).view(torch.uint8)
+        out[name] = codes.contiguous()
+        out["descale_" + name] = ds
+    return out
+
+
+def make_fp8(w: Workload, *, B=None, Hq=None, Hkv=None, N=None, d=None, seed=None):
+    """``draw_fp8`` for workload ``w`` (optionally with shapes overridden)."""
+    return draw_fp8(w.B if B is None else B, w.Hq if Hq is None else Hq,
+                    w.Hkv if Hkv is None else Hkv, w.N if N is None else N,
+                    w.d if d is None else d, w.seed if seed is None else seed, w.q_mul)
 
 
 def as_f64(t):
