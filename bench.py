@@ -307,7 +307,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": (1 + 2 + (2 if w.d == 256 else 1) + 1) * args.steps,
         "clocks": clk,
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if dist is not None:
         dist.destroy_process_group()
@@ -315,8 +315,9 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(out), flush=True)
 
 
-def run_inference(args, rank, world, local_rank):
-    """Forward only, split-KV path, on an inference-shaped workload."""
+def run_forward_only(args, rank, world, local_rank):
+    """Forward only: the split-KV path on an inference-shaped workload, or the
+    E4M3 forward on an e4m3 workload."""
     import torch
     import attn_inputs
     import exact_io_aware_50_b200 as F
@@ -330,22 +331,29 @@ def run_inference(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = attn_inputs.BY_NAME[args.workload]
     fwd_f, _ = flops(w)
-    x = attn_inputs.make(w, seed=w.seed + 1000 * rank)
+    fp8 = w.dtype == "e4m3"
+    x = (attn_inputs.make_fp8 if fp8 else attn_inputs.make)(w, seed=w.seed + 1000 * rank)
     g = {k: x[k].to(dev) for k in ("q", "k", "v")}
     B, Hq, Hkv, Nq, Nk, d = w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d
-    splits = F.fa_fwd_splitkv_num_splits(B, Hq, Nq, Nk, d)
-    o = torch.empty_like(g["q"])
+    splits = 1 if fp8 else F.fa_fwd_splitkv_num_splits(B, Hq, Nq, Nk, d)
+    o = torch.empty(B, Hq, Nq, d, device=dev, dtype=torch.bfloat16)
     lse = torch.empty(B, Hq, Nq, device=dev, dtype=torch.float32)
     ws = torch.empty(max(F.fa_fwd_splitkv_workspace_size(B, Hq, Nq, d, splits), 1), device=dev,
                      dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        st = F.fa_fwd_splitkv(g["q"].data_ptr(), g["k"].data_ptr(), g["v"].data_ptr(),
-                              o.data_ptr(), lse.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
-                              w.scale, w.causal, splits, stream.cuda_stream)
+        if fp8:
+            st = F.fa_fwd_fp8(g["q"].data_ptr(), g["k"].data_ptr(), g["v"].data_ptr(),
+                              o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, d, w.scale,
+                              x["descale_q"], x["descale_k"], x["descale_v"], w.causal,
+                              stream.cuda_stream)
+        else:
+            st = F.fa_fwd_splitkv(g["q"].data_ptr(), g["k"].data_ptr(), g["v"].data_ptr(),
+                                  o.data_ptr(), lse.data_ptr(), ws.data_ptr(), B, Hq, Hkv, Nq, Nk,
+                                  d, w.scale, w.causal, splits, stream.cuda_stream)
         if st != 0:
-            raise RuntimeError(f"fa_fwd_splitkv: {F.fa_strerror(st)}")
+            raise RuntimeError(f"{'fa_fwd_fp8' if fp8 else 'fa_fwd_splitkv'}: {F.fa_strerror(st)}")
 
     for _ in range(args.warmup):
         step()
@@ -389,25 +397,41 @@ def run_inference(args, rank, world, local_rank):
     ms = total_ms / args.steps
     burst, _, _, src = measured_peaks()
     value = whole_job_tflops(world, fwd_f, ms)
+    achieved = fwd_f / (ms * 1e-3) / 1e12
+    if fp8:
+        # e4m3 dense peak: the measured bf16 burst times the nominal ratio
+        # (4.5 / 2.25 PFLOP/s dense)
+        peak, peak_src = 2.0 * burst, f"{src} bf16 dense burst x 2 (nominal e4m3/bf16 ratio)"
+        metric = "attention forward TFLOP/s (FP8 e4m3 inputs, bf16 output)"
+        data = "synthetic (seeded N(0,1) float32 quantised per tensor to e4m3, shapes of the workload)"
+        l2 = "inputs larger than L2 (no flush): q,k,v e4m3 96 MiB + o bf16 64 MiB"
+        kernel = "fa_fwd_fp8"
+    else:
+        peak, peak_src = burst, f"{src} bf16 dense burst (MEASURED_PEAKS.json)"
+        metric = "attention forward TFLOP/s (BF16, split-KV inference shape)"
+        data = "synthetic (seeded N(0,1) bf16, shapes of the workload)"
+        l2 = "K/V 64 MiB (L2-resident between steps)"
+        kernel = "fa_fwd_splitkv (pieces + merge)"
     out = {
-        "metric": "attention forward TFLOP/s (BF16, split-KV inference shape)",
+        "metric": metric,
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
-        "config": dict(config_dict(w, world, "K/V 64 MiB (L2-resident between steps)"),
-                       num_splits=splits),
-        "roofline": {"bound": "tensor", "kernel": "fa_fwd_splitkv (pieces + merge)",
-                     "achieved": round(fwd_f / (ms * 1e-3) / 1e12, 2), "peak": burst,
-                     "peak_source": f"{src} bf16 dense burst (MEASURED_PEAKS.json)",
-                     "unit": "TFLOP/s", "frac": round(fwd_f / (ms * 1e-3) / 1e12 / burst, 4),
-                     "traffic": None},
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
+        "data": data,
+        "config": dict(config_dict(w, world, l2), num_splits=splits),
+        "roofline": {"bound": "tensor", "kernel": kernel,
+                     "achieved": round(achieved, 2), "peak": round(peak, 2),
+                     "peak_source": peak_src,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": load_traffic(w.name, "fa_fwd_fp8") if fp8 else None},
         "e2e": {"value": round(whole_job_tflops(world, fwd_f, e2e_ms), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": (2 if splits > 1 else 1) * args.steps,
         "clocks": clk,
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if dist is not None:
         dist.destroy_process_group()
     if rank == 0:
@@ -459,15 +483,25 @@ def cpu_baseline(w, seconds):
     import numpy as np
     import attn_inputs
     import oracle
-    x = attn_inputs.make(w, B=1, Hq=w.Hq // w.Hkv, Hkv=1)  # one key/value group of batch 0
-    q, k, v, do = (attn_inputs.as_f64(x[n]) for n in ("q", "k", "v", "do"))
+    import oracle.fp8
+    fp8 = w.dtype == "e4m3"
+    if fp8:
+        x = attn_inputs.make_fp8(w, B=1, Hq=w.Hq // w.Hkv, Hkv=1)
+        q, k, v = (x[n].numpy() for n in ("q", "k", "v"))
+    else:
+        x = attn_inputs.make(w, B=1, Hq=w.Hq // w.Hkv, Hkv=1)  # one key/value group of batch 0
+        q, k, v, do = (attn_inputs.as_f64(x[n]) for n in ("q", "k", "v", "do"))
     heads = 0
     t0 = time.perf_counter()
     g = w.Hq // w.Hkv
     off = w.Nk - w.Nq if w.causal else 0     # bottom-right alignment when Nq < Nk
     while True:
         h = heads % g
-        oracle.forward(q[:, h:h + 1], k, v, w.scale, w.causal, off)
+        if fp8:
+            oracle.fp8.fp8_forward(q[:, h:h + 1], k, v, x["descale_q"], x["descale_k"],
+                                   x["descale_v"], w.scale, w.causal)
+        else:
+            oracle.forward(q[:, h:h + 1], k, v, w.scale, w.causal, off)
         if w.backward:
             oracle.backward(q[:, h:h + 1], k, v, do[:, h:h + 1], w.scale, w.causal)
         heads += 1
@@ -504,7 +538,7 @@ def run_reference(args, rank, world):
         samples.append(cb)
     value = statistics.median(vals)
     fwd_f, bwd_f = flops(w)
-    ms = (fwd_f + bwd_f) / (value * 1e12) * 1e3
+    ms = (fwd_f + (bwd_f if w.backward else 0.0)) / (value * 1e12) * 1e3
     cb = dict(samples[-1])
     cb["value"] = value
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
@@ -539,8 +573,8 @@ def main():
     w = attn_inputs.BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, rank, world)
-    elif not w.backward and w.Nq < w.Nk:
-        run_inference(args, rank, world, local_rank)
+    elif not w.backward and (w.Nq < w.Nk or w.dtype == "e4m3"):
+        run_forward_only(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

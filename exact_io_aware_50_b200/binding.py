@@ -24,7 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libfa.so")
 _lib = None
 
-EXPORTS = ("fa_fwd", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_splitkv",
+EXPORTS = ("fa_fwd", "fa_fwd_fp8", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_splitkv",
            "fa_fwd_splitkv_num_splits",
            "fa_fwd_splitkv_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prep",
            "fa_bwd_dkdv",
@@ -53,6 +53,8 @@ def lib():
         L.fa_fwd_f32.argtypes = [P] * 5 + dims
         L.fa_fwd_f32.restype = I
         U64 = ctypes.c_ulonglong
+        L.fa_fwd_fp8.argtypes = [P] * 5 + [I, I, I, I, I, F, F, F, F, I, P]
+        L.fa_fwd_fp8.restype = I
         L.fa_fwd_dropout.argtypes = [P] * 5 + [I, I, I, I, I, I, F, I, F, U64, U64, P]
         L.fa_fwd_dropout.restype = I
         L.fa_bwd_dropout.argtypes = [P] * 10 + [I, I, I, I, I, I, F, I, F, U64, U64, P]
@@ -90,6 +92,12 @@ def lib():
 # ----------------------------------------------------------------- raw ABI
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
     return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, int(causal), stream)
+
+
+def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, descale_q, descale_k, descale_v, causal,
+               stream=0):
+    return lib().fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, float(descale_q),
+                            float(descale_k), float(descale_v), int(causal), stream)
 
 
 def fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, p_drop, seed, offset,
@@ -228,6 +236,26 @@ def forward_splitkv(q, k, v, scale=None, causal=False, num_splits=None, workspac
     _check(fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
                           workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits,
                           _stream(q)), "fa_fwd_splitkv")
+    return o, L
+
+
+def forward_fp8(q, k, v, descale_q, descale_k, descale_v, scale=None, causal=False):
+    """O (bf16), L from E4M3 inputs (fa_fwd_fp8).  q, k, v: contiguous CUDA
+    tensors of dtype float8_e4m3fn or uint8 (the codes); descale_*: the
+    per-tensor dequantisation factors."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
+    if Nq != Nk:
+        raise ValueError("fa_fwd_fp8 takes Nq == Nk")
+    scale = d ** -0.5 if scale is None else float(scale)
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise ValueError("inputs must be contiguous float8_e4m3fn (or uint8) CUDA tensors")
+    o = torch.empty(q.shape, device=q.device, dtype=torch.bfloat16)
+    L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
+    _check(fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                      B, Hq, Hkv, Nq, d, scale, descale_q, descale_k, descale_v, causal,
+                      _stream(q)), "fa_fwd_fp8")
     return o, L
 
 

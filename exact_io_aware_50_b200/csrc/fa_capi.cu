@@ -268,6 +268,29 @@ FA_EXPORT int fa_fwd_dropout(const void *q, const void *k, const void *v, void *
   return fa::launch_fwd_bf16_sm100(a);
 }
 
+FA_EXPORT int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
+                         int B, int Hq, int Hkv, int N, int d, float scale, float descale_q,
+                         float descale_k, float descale_v, int causal, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  const float ds[3] = {descale_q, descale_k, descale_v};
+  for (float x : ds)
+    if (!(x > 0.f) || !isfinite(x)) return FA_ERR_INVALID_ARG;
+  int st = fa::check_sizes(B, Hq, Hkv, N, N, d, scale, causal);
+  if (st) return st;
+  if (d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!fa::aligned16(q) || !fa::aligned16(k) || !fa::aligned16(v) || !fa::aligned16(o) ||
+      !fa::aligned16(lse))
+    return FA_ERR_ALIGNMENT;
+  AttnArgs a;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = N; a.Nk = N; a.d = d;
+  a.scale = scale; a.causal = causal ? 1 : 0; a.stream = (cudaStream_t)stream;
+  a.descale_q = descale_q; a.descale_k = descale_k; a.descale_v = descale_v;
+  return fa::launch_fwd_e4m3_sm100(a);
+}
+
 FA_EXPORT int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o,
                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
                              void *workspace, int B, int Hq, int Hkv, int Nq, int Nk, int d,

@@ -44,6 +44,16 @@
 // a row); the row sum uses the undropped P and the epilogue scales O by
 // 1 / (1 - p).
 //
+// E4M3 instances (C::F8): Q, K, V are one-byte OCP E4M3 codes with one
+// dequantisation factor each.  S = Q K^T runs as tcgen05 kind::f8f6f4 (K = 32
+// per instruction), the Q and K factors fold into the softmax scale, P goes
+// to TMEM as e4m3 (four per column) for the P V product (V MN-major, as in
+// the bf16 path), and the V factor joins the final 1 / l.  P is stored as
+// 2^4 * 2^(x - m) with the rescale threshold at 2^4, so stored values stay at
+// or below 256 (e4m3 saturates at 448); the shift cancels in O / l and is
+// taken out of L.  The wiki's FlashAttention-3 paragraph names FP8 as one of
+// FA3's Hopper features and defines nothing further.
+//
 // MMA issue order per block j (two tiles): PV0(j), S0(j+1), PV1(j), S1(j+1):
 // the softmax of one tile overlaps the tensor-core work of the other.
 // tcgen05 ops of one thread complete in issue order, and tcgen05.commit
@@ -70,10 +80,23 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // than MUFU alone, so the exponential unit is not what bounds this kernel.
 constexpr bool kPolyExp = FA_FWD_POLY_EXP != 0;
 
-template <int D_, int NT_, int BN_, int STAGES_>
+// ES: bytes per Q/K/V element, 2 for bf16, 1 for e4m3.  Tiles are laid out in
+// bytes (128-byte swizzled rows), so an e4m3 d = 128 tile has the shape of a
+// bf16 d = 64 one.
+template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2>
 struct FwdCfg {
-  static constexpr int D = D_, NT = NT_, BN = BN_, STAGES = STAGES_;
-  static constexpr int DCH = D / 64;                      // 128-byte column chunks
+  static constexpr int D = D_, NT = NT_, BN = BN_, STAGES = STAGES_, ES = ES_;
+  static constexpr bool F8 = ES == 1;
+  static constexpr int DCH = D * ES / 128;                // 128-byte column chunks
+  static constexpr int CH_ELEMS = 128 / ES;               // elements per chunk (TMA box width)
+  static constexpr int MMA_K = 32 / ES;                   // K of one MMA: 32 bytes of a row
+  static constexpr int S_STEPS = D / MMA_K;               // MMAs per S tile
+  static constexpr int PV_STEPS = BN / MMA_K;             // MMAs per P V
+  // P is stored as 2^P_SHIFT * 2^(x - m): for e4m3 that keeps the largest
+  // stored value (2^(P_SHIFT + RESCALE)) inside the format's 448 and lifts
+  // small values out of its subnormal range.
+  static constexpr float P_SHIFT = F8 ? 4.f : 0.f;
+  static constexpr float RESCALE = F8 ? 4.f : kRescaleThreshold;
   static constexpr int Q_CHUNK = BM * 128;                // bytes of one chunk of a Q tile
   static constexpr int KV_CHUNK = BN * 128;
   static constexpr int Q_TILE = Q_CHUNK * DCH;
@@ -95,6 +118,8 @@ struct FwdCfg {
   static_assert(TM_COLS_USED <= TM_ALLOC, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN == 128, "softmax path assumes 128 columns per block");
+  static_assert(ES == 1 || ES == 2, "bf16 or e4m3 operands");
+  static_assert(D * ES % 128 == 0, "whole 128-byte rows per chunk");
 };
 
 struct FwdParams {
@@ -109,9 +134,9 @@ struct FwdParams {
   float *o_part;     // splits > 1: [splits][B*Hq][Nq][D] normalised partial O
   float *l_part;     // splits > 1: [splits][B*Hq][Nq] partial log-sum-exp (natural log)
   // dropout on P (DROP kernels): keep when the Philox word >= drop_thr; kept
-  // values are scaled by drop_scale = 1 / (1 - p) in the epilogue
+  // values are scaled by 1 / (1 - p) (o_scale) in the epilogue
   uint32_t drop_thr, seed_lo, seed_hi, drop_off;
-  float drop_scale;
+  float o_scale;     // epilogue factor on O: 1 / (1 - p) with dropout, the V descale for e4m3
   unsigned *err;
 };
 
@@ -119,6 +144,7 @@ template <class C, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  static_assert(!(DROP && C::F8), "dropout is built for the bf16 forward only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -226,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < C::NT; ++t)
           for (int c = 0; c < C::DCH; ++c)
             tma_load_3d(sbase + C::OFF_Q + t * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(B_QFULL),
-                        c * 64, U.q_start + t * BM, U.bh);
+                        c * C::CH_ELEMS, U.q_start + t * BM, U.bh);
         last_q_phase = uq & 1;
         for (int j = 0; j < U.nkb && ok; ++j, ++g) {
           const int s = g % C::STAGES;
@@ -236,14 +262,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar(B_KFULL + s), C::KV_TILE);
           for (int c = 0; c < C::DCH; ++c)
             tma_load_3d(sbase + C::OFF_K + s * C::KV_TILE + c * C::KV_CHUNK, &tmK,
-                        bar(B_KFULL + s), c * 64, (U.j0 + j) * C::BN, U.bh_kv);
+                        bar(B_KFULL + s), c * C::CH_ELEMS, (U.j0 + j) * C::BN, U.bh_kv);
           last_k_phase[s] = ph;
           ok = bounded_wait(bar(B_VEMPTY + s), ph ^ 1, wc);
           if (!ok) break;
           mbar_arrive_expect_tx(bar(B_VFULL + s), C::KV_TILE);
           for (int c = 0; c < C::DCH; ++c)
             tma_load_3d(sbase + C::OFF_V + s * C::KV_TILE + c * C::KV_CHUNK, &tmV,
-                        bar(B_VFULL + s), c * 64, (U.j0 + j) * C::BN, U.bh_kv);
+                        bar(B_VFULL + s), c * C::CH_ELEMS, (U.j0 + j) * C::BN, U.bh_kv);
           last_v_phase[s] = ph;
         }
         ++uq;
@@ -260,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t IDESC_S = idesc_bf16(BM, C::BN, 0, 0);
-    constexpr uint32_t IDESC_PV = idesc_bf16(BM, C::D, 0, 1);
+    constexpr uint32_t IDESC_S = C::F8 ? idesc_e4m3(BM, C::BN, 0, 0) : idesc_bf16(BM, C::BN, 0, 0);
+    constexpr uint32_t IDESC_PV = C::F8 ? idesc_e4m3(BM, C::D, 0, 1) : idesc_bf16(BM, C::D, 0, 1);
     // Descriptors are built once; each MMA offsets a base descriptor.
     const uint64_t dq0 = sw128_desc(sbase + C::OFF_Q, 16, 1024);
     const uint64_t dk0 = sw128_desc(sbase + C::OFF_K, 16, 1024);
@@ -270,20 +296,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qa = desc_add(dq0, t * C::Q_TILE);
       const uint64_t kb = desc_add(dk0, s * C::KV_TILE);
 #pragma unroll
-      for (int kk = 0; kk < C::D / 16; ++kk) {
+      for (int kk = 0; kk < C::S_STEPS; ++kk) {
         const uint32_t off = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
         const uint32_t offk = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
-        mma_ss(tmem + C::TM_S + t * C::BN, desc_add(qa, off), desc_add(kb, offk), IDESC_S,
-               kk > 0);
+        if constexpr (C::F8)
+          mma_ss_f8(tmem + C::TM_S + t * C::BN, desc_add(qa, off), desc_add(kb, offk), IDESC_S,
+                    kk > 0);
+        else
+          mma_ss(tmem + C::TM_S + t * C::BN, desc_add(qa, off), desc_add(kb, offk), IDESC_S,
+                 kk > 0);
       }
     };
     auto issue_PV = [&](int t, int s, bool first) {
       const uint64_t vb = desc_add(dv0, s * C::KV_TILE);
       const uint32_t pcol = tmem + C::TM_S + t * C::BN + C::BN / 2;
 #pragma unroll
-      for (int kk = 0; kk < C::BN / 16; ++kk) {
-        mma_ts(tmem + C::TM_O + t * C::D, pcol + kk * 8, desc_add(vb, kk * 16 * 128),
-               IDESC_PV, (!first) || kk > 0);
+      for (int kk = 0; kk < C::PV_STEPS; ++kk) {
+        // MMA_K keys of P = 8 TMEM columns (two bf16 or four e4m3 per column);
+        // MMA_K rows of the MN-major V tile
+        if constexpr (C::F8)
+          mma_ts_f8(tmem + C::TM_O + t * C::D, pcol + kk * 8, desc_add(vb, kk * C::MMA_K * 128),
+                    IDESC_PV, (!first) || kk > 0);
+        else
+          mma_ts(tmem + C::TM_O + t * C::D, pcol + kk * 8, desc_add(vb, kk * C::MMA_K * 128),
+                 IDESC_PV, (!first) || kk > 0);
       }
     };
     // The whole role runs in lane 0; the other lanes wait at the end.
@@ -419,12 +455,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float alpha = 1.f;
         if (j == 0) {
           m_run = m_new;
-        } else if (__any_sync(0xffffffffu, m_new - m_run > kRescaleThreshold)) {
+        } else if (__any_sync(0xffffffffu, m_new - m_run > C::RESCALE)) {
           rescale = true;
           alpha = fast_exp2(m_run - m_new);
           m_run = m_new;
         }
-        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        const float m_use = ((m_run == -INFINITY) ? 0.f : m_run) - C::P_SHIFT;
         // p = 2^(s * scale * log2e - m) on MUFU (exp2_poly for one column in
         // four when FA_FWD_POLY_EXP is set); row sum in four independent
         // partials over the undropped p; with dropout, P in TMEM keeps only the
@@ -448,11 +484,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     (uint32_t)bh, p.drop_off, p.seed_lo, p.seed_hi);
               const uint32_t w0 = (e & 1) ? rnd.z : rnd.x, w1 = (e & 1) ? rnd.w : rnd.y;
               pk[e] = pack_bf16x2(w0 >= p.drop_thr ? p0 : 0.f, w1 >= p.drop_thr ? p1 : 0.f);
+            } else if constexpr (C::F8) {
+              // four e4m3 codes per column: keys 2e, 2e + 1 in the low half
+              // of word e / 2 for even e, in the high half for odd e
+              const uint32_t h = pack_e4m3x2(p0, p1);
+              pk[e >> 1] = (e & 1) ? (pk[e >> 1] | (h << 16)) : h;
             } else {
               pk[e] = pack_bf16x2(p0, p1);
             }
           }
-          tmem_st16(tP + c * 16, pk);
+          if constexpr (C::F8)
+            tmem_st8(tP + c * 8, *reinterpret_cast<const uint32_t(*)[8]>(pk));
+          else
+            tmem_st16(tP + c * 16, pk);
         }
         const float rowsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
         l_run = l_run * alpha + rowsum;
@@ -498,10 +542,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(bar(B_OEMPTY + t));   // O_t read out: the next unit may overwrite it
-        if (live) p.l_part[prow] = empty ? -INFINITY : (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        if (live)
+          p.l_part[prow] =
+              empty ? -INFINITY : (m_run + __log2f(l_run) - C::P_SHIFT) * 0.69314718055994531f;
       } else if (ok) {
         tc_fence_after();
-        const float inv_l = (DROP ? p.drop_scale : 1.f) / l_run;
+        const float inv_l = p.o_scale / l_run;
         const bool live = row < p.Nq;
         __nv_bfloat16 *orow = p.o + ((size_t)bh * p.Nq + (live ? row : 0)) * C::D;
   #pragma unroll 1
@@ -523,7 +569,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(bar(B_OEMPTY + t));   // O_t read out: the next unit may overwrite it
-        if (live) p.o_lse[(size_t)bh * p.Nq + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        if (live)
+          p.o_lse[(size_t)bh * p.Nq + row] =
+              (m_run + __log2f(l_run) - C::P_SHIFT) * 0.69314718055994531f;
       }
       g += U.nkb;
       ++uq;
@@ -538,15 +586,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// [heads][rows][d] tensor of `es`-byte elements (2: bf16, 1: e4m3 bytes);
+// box = one 128-byte chunk of box_rows rows, 128-byte swizzle.
 bool make_map(CUtensorMap *m, const void *base, int rows_per_head, int heads, int d,
-              int box_rows) {
+              int box_rows, int es = 2) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows_per_head, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows_per_head * d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)d * es, (cuuint64_t)rows_per_head * d * es};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+  const CUtensorMapDataType dt = es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -554,9 +605,10 @@ bool make_map(CUtensorMap *m, const void *base, int rows_per_head, int heads, in
 template <class C>
 int run_fwd(const AttnArgs &a) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, a.q, a.Nq, a.B * a.Hq, C::D, BM) ||
-      !make_map(&mk, a.k, a.Nk, a.B * a.Hkv, C::D, C::BN) ||
-      !make_map(&mv, a.v, a.Nk, a.B * a.Hkv, C::D, C::BN))
+  if (C::F8 && (a.drop_thr != 0 || a.splits > 1)) return 2;   // e4m3: plain forward only
+  if (!make_map(&mq, a.q, a.Nq, a.B * a.Hq, C::D, BM, C::ES) ||
+      !make_map(&mk, a.k, a.Nk, a.B * a.Hkv, C::D, C::BN, C::ES) ||
+      !make_map(&mv, a.v, a.Nk, a.B * a.Hkv, C::D, C::BN, C::ES))
     return 5;
   FwdParams p;
   p.o_lse = a.lse;
@@ -564,7 +616,9 @@ int run_fwd(const AttnArgs &a) {
   p.Hq = a.Hq; p.Hkv = a.Hkv; p.Nq = a.Nq; p.Nk = a.Nk;
   p.nqb = (a.Nq + C::NT * BM - 1) / (C::NT * BM);
   p.BH = a.B * a.Hq;
-  p.scale_log2 = a.scale * 1.4426950408889634f;
+  // e4m3: the Q and K descales fold into the score scale
+  p.scale_log2 = (float)((double)a.scale * (C::F8 ? (double)a.descale_q * a.descale_k : 1.0) *
+                         1.4426950408889634);
   p.causal = a.causal;
   p.causal_off = a.causal_off;
   p.splits = a.splits;
@@ -575,10 +629,12 @@ int run_fwd(const AttnArgs &a) {
   p.seed_lo = (uint32_t)a.seed;
   p.seed_hi = (uint32_t)(a.seed >> 32);
   p.drop_off = (uint32_t)a.drop_offset;
-  p.drop_scale = a.drop_scale;
+  p.o_scale = a.drop_thr != 0 ? a.drop_scale : (C::F8 ? a.descale_v : 1.f);
   p.err = a.err;
   if (a.drop_thr != 0 && a.splits > 1) return 2;   // dropout only in the plain forward
-  auto kern = a.drop_thr != 0 ? fwd_kernel<C, true> : fwd_kernel<C, false>;
+  auto kern = fwd_kernel<C, false>;
+  if constexpr (!C::F8)
+    if (a.drop_thr != 0) kern = fwd_kernel<C, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return 5;
@@ -690,6 +746,14 @@ int launch_fwd_splitkv_bf16_sm100(const AttnArgs &a) {
     case 64: return run_combine<64>(a);
     case 128: return run_combine<128>(a);
     case 256: return run_combine<256>(a);
+    default: return 2;
+  }
+}
+
+int launch_fwd_e4m3_sm100(const AttnArgs &a) {
+  switch (a.d) {
+    case 128: return run_fwd<FwdCfg<128, 2, 128, 4, 1>>(a);
+    case 256: return run_fwd<FwdCfg<256, 1, 128, 2, 1>>(a);
     default: return 2;
   }
 }

@@ -26,6 +26,8 @@ struct AttnArgs {
   uint32_t drop_thr = 0;
   float drop_scale = 1.f;
   unsigned long long seed = 0, drop_offset = 0;
+  // e4m3 forward: per-tensor dequantisation factors (tensor = factor * code value)
+  float descale_q = 1.f, descale_k = 1.f, descale_v = 1.f;
   cudaStream_t stream = nullptr;
   unsigned *err = nullptr;      // device error word
 };
@@ -63,6 +65,7 @@ int launch_fwd_f32(const AttnArgs &a);
 int launch_bwd_f32(const AttnArgs &a);
 int launch_fwd_bf16_sm100(const AttnArgs &a);
 int launch_fwd_splitkv_bf16_sm100(const AttnArgs &a);   // pieces + merge (splits > 1)
+int launch_fwd_e4m3_sm100(const AttnArgs &a);   // e4m3 Q/K/V, bf16 O (d = 128, 256)
 int launch_bwd_bf16_sm100(const AttnArgs &a);   // all three stages
 int launch_bwd_prep_bf16(const AttnArgs &a);     // D + zeroed dQ accumulator
 int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a);

@@ -134,6 +134,35 @@ int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, c
                    fa_stream_t stream);
 
 /*
+ * fa_fwd_fp8 -- attention forward on FP8 inputs.  The wiki's FlashAttention-3
+ * paragraph ("FlashAttention", newton.com.tw) names low-precision FP8 as one
+ * of the Hopper features FA3 uses and defines nothing further; this entry
+ * point reads it as: Q, K, V hold OCP FP8 E4M3 codes (one byte per element:
+ * sign, 4 exponent bits with bias 7, 3 mantissa bits; largest finite 448),
+ * each tensor with one dequantisation factor, so the tensors meant are
+ * descale_q * Q^, descale_k * K^, descale_v * V^ (code values Q^ ...), and
+ *     O = softmax(scale * (descale_q Q^)(descale_k K^)^T [+ causal]) (descale_v V^),
+ *     L = log-sum-exp of the scaled scores (natural log, float32),
+ * the same quantity as fa_fwd computes for those tensors.  S accumulates in
+ * float32 on the tensor cores; P is rounded to e4m3 for the P V product
+ * (after scaling so its values lie in [2^-10, 256] or flush below, a relative
+ * error of at most 2^-4 per element), O is accumulated in float32 and
+ * written as bf16.
+ *
+ * q [B, Hq, N, d], k and v [B, Hkv, N, d]: E4M3 codes, contiguous, 16-byte
+ * aligned; o [B, Hq, N, d] bf16 and lse [B, Hq, N] float32 written by the
+ * call (caller-owned device memory).  Nq = Nk = N; causal is top-left.
+ * descale_*: finite and > 0 (else FA_ERR_INVALID_ARG).  d = 128 or 256
+ * (FA_ERR_UNSUPPORTED otherwise).  Other size rules and errors as fa_fwd.
+ * Code values that are NaN (S.1111.111) give NaN outputs for the rows they
+ * reach.
+ */
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
+               int B, int Hq, int Hkv, int N, int d, float scale,
+               float descale_q, float descale_k, float descale_v, int causal,
+               fa_stream_t stream);
+
+/*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd and fa_bwd_f32
  * need (float32 throughout): the per-row vector D = rowsum(dO * O) and the
  * per-row base-2 log-sum-exp used by the backward, each padded to a multiple

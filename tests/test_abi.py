@@ -155,6 +155,28 @@ def test_dropout_argument_errors():
     assert fwd(0.1, ptrs=(FAKE + 2,) + (FAKE,) * 4) == F.FA_ERR_ALIGNMENT
 
 
+def test_fp8_argument_errors():
+    def fwd(dq=0.5, dk=0.5, dv=0.5, d=128, ptrs=(FAKE,) * 5, scale=0.125, causal=0, B=1):
+        return F.fa_fwd_fp8(*ptrs, B, 2, 1, 8, d, scale, dq, dk, dv, causal)
+
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        assert fwd(dq=bad) == F.FA_ERR_INVALID_ARG
+        assert fwd(dk=bad) == F.FA_ERR_INVALID_ARG
+        assert fwd(dv=bad) == F.FA_ERR_INVALID_ARG
+    assert fwd(scale=0.0) == F.FA_ERR_INVALID_ARG
+    assert fwd(B=0) == F.FA_ERR_INVALID_ARG
+    for i in range(5):
+        ptrs = [FAKE] * 5
+        ptrs[i] = 0
+        assert fwd(ptrs=tuple(ptrs)) == F.FA_ERR_INVALID_ARG
+    for d in (64, 96, 192, 512):
+        assert fwd(d=d) == F.FA_ERR_UNSUPPORTED       # e4m3 forward: d = 128, 256
+    for i in range(5):
+        ptrs = [FAKE] * 5
+        ptrs[i] = FAKE + 8
+        assert fwd(ptrs=tuple(ptrs)) == F.FA_ERR_ALIGNMENT
+
+
 def test_size_limits():
     """Sizes past the kernels' index arithmetic are refused before any launch."""
     f = F.fa_fwd
