@@ -1,14 +1,15 @@
-// fa_fwd_sm100.cu -- BF16 attention forward for sm_100a: TMA-fed shared-memory
-// ring, tcgen05 MMA with TMEM accumulators, one softmax thread per query row.
+// fa_fwd_sm100.cu -- BF16 and E4M3 attention forward for sm_100a: TMA-fed
+// shared-memory ring, tcgen05 MMA with TMEM accumulators, one softmax thread
+// per query row.
 //
 // Method (FlashAttention blog, sections 2-4; CSDN FlashAttention-1 tutorial,
 // section 3): Q is cut into 128-row tiles (outer loop, one or two tiles per
 // CTA), K and V into 128-row blocks (inner loop).  For every block:
 //     S = Q K_j^T                     tcgen05, bf16 x bf16 -> f32 in TMEM
 //     m_new = max(m, rowmax(S*scale)) softmax thread of the row
-//     P = exp(S*scale - m)            written back to TMEM as bf16
+//     P = exp(S*scale - m)            to shared memory (or TMEM) as bf16
 //     l = e^{m_old - m} l + rowsum(P)
-//     O~ = e^{m_old - m} O~ + P V_j   tcgen05, P from TMEM, V from SMEM
+//     O~ = e^{m_old - m} O~ + P V_j   tcgen05, P and V from SMEM (or P from TMEM)
 // and after the last block O = O~ / l, L = m + ln(l) (deferred
 // normalisation, blog section 4.1).  The rescale of O~ is skipped while the
 // running max has grown by less than 2^8 (in base-2 units): p values then stay
@@ -39,26 +40,36 @@
 // causal mask may be bottom-right aligned there (key j hidden from query i
 // when j > i + Nk - Nq).
 //
-// Dropout (DROP instances): P written to TMEM keeps only the elements whose
+// Dropout (DROP instances): the stored P keeps only the elements whose
 // Philox4x32-10 word is >= floor(p 2^32) (one counter per four key columns of
 // a row); the row sum uses the undropped P and the epilogue scales O by
 // 1 / (1 - p).
 //
 // E4M3 instances (C::F8): Q, K, V are one-byte OCP E4M3 codes with one
 // dequantisation factor each.  S = Q K^T runs as tcgen05 kind::f8f6f4 (K = 32
-// per instruction), the Q and K factors fold into the softmax scale, P goes
-// to TMEM as e4m3 (four per column) for the P V product (V MN-major, as in
-// the bf16 path), and the V factor joins the final 1 / l.  P is stored as
+// per instruction), the Q and K factors fold into the softmax scale, P is
+// stored as e4m3 (one byte per key; four per TMEM column in the TMEM form)
+// for the P V product (V MN-major, as in the bf16 path), and the V factor
+// joins the final 1 / l.  P is stored as
 // 2^4 * 2^(x - m) with the rescale threshold at 2^4, so stored values stay at
 // or below 256 (e4m3 saturates at 448); the shift cancels in O / l and is
 // taken out of L.  The wiki's FlashAttention-3 paragraph names FP8 as one of
 // FA3's Hopper features and defines nothing further.
 //
-// MMA issue order per block j (two tiles): PV0(j), S0(j+1), PV1(j), S1(j+1):
-// the softmax of one tile overlaps the tensor-core work of the other.
-// tcgen05 ops of one thread complete in issue order, and tcgen05.commit
-// arrives after all earlier ops, so "S_t(j+1) ready" also means "PV_t(j)
-// done": the softmax thread may rescale O~ in TMEM right then.
+// Two pipelines (FwdCfg::PS):
+// * P through shared memory (PS): the softmax thread reads S_t(j) out of
+//   TMEM and arrives on s_empty; the MMA issuer then starts S_t(j+1) in the
+//   same columns while block j's exponentials run.  P_t(j) goes to a K-major
+//   128-byte-swizzled shared-memory tile once P_t(j-1) V_{j-1} has released
+//   it (p_empty, which also orders the rare O~ rescale after that MMA), and
+//   P_t(j) V_j runs SMEM x SMEM.  Issue order per block: S0(j+1), S1(j+1),
+//   PV0(j), PV1(j); the producer loads K one block ahead of V.
+// * P in TMEM (d = 256 bf16): P overwrites the upper half of S_t's columns;
+//   issue order PV0(j), S0(j+1), PV1(j), S1(j+1), so the softmax of one tile
+//   overlaps the tensor-core work of the other.  tcgen05 ops of one thread
+//   complete in issue order, and tcgen05.commit arrives after all earlier
+//   ops, so "S_t(j+1) ready" also means "PV_t(j) done": the softmax thread
+//   may rescale O~ in TMEM right then.
 #include <math.h>
 
 #include "common.cuh"
