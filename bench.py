@@ -451,21 +451,30 @@ def load_traffic(workload, kernel):
         ent = d.get(workload, {}).get(kernel)
         if not ent:
             return None
-        if ent.get("source_sha") != source_sha():
+        if ent.get("source_sha") != source_sha(KERNEL_SOURCES.get(kernel)):
             return None
         return ent.get("bytes_per_launch")
     except (OSError, ValueError):
         return None
 
 
-def source_sha():
-    """Hash of the kernel sources with comments and blank lines removed, so a
-    comment edit does not invalidate recorded counters but a code edit does."""
+# The sources each recorded kernel is compiled from.
+KERNEL_SOURCES = {
+    "fa_fwd": ("common.cuh", "fa_fwd_sm100.cu", "launch.h"),
+    "fa_fwd_fp8": ("common.cuh", "fa_fwd_sm100.cu", "launch.h"),
+    "fa_bwd_dkdv": ("common.cuh", "fa_bwd_sm100.cu", "launch.h"),
+}
+
+
+def source_sha(files=None):
+    """Hash of the given kernel source files (default: all of them) with
+    comments and blank lines removed, so a comment edit does not invalidate
+    recorded counters but a code edit does."""
     import hashlib
     import re
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "exact_io_aware_50_b200", "csrc")
-    for f in sorted(os.listdir(cs)):
+    for f in sorted(files or os.listdir(cs)):
         with open(os.path.join(cs, f)) as fh:
             text = fh.read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
