@@ -144,10 +144,11 @@ int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, c
  *     O = softmax(scale * (descale_q Q^)(descale_k K^)^T [+ causal]) (descale_v V^),
  *     L = log-sum-exp of the scaled scores (natural log, float32),
  * the same quantity as fa_fwd computes for those tensors.  S accumulates in
- * float32 on the tensor cores; P is rounded to e4m3 for the P V product
- * (after scaling so its values lie in [2^-10, 256] or flush below, a relative
- * error of at most 2^-4 per element), O is accumulated in float32 and
- * written as bf16.
+ * float32 on the tensor cores; P is rounded to e4m3 for the P V product,
+ * stored as 2^4 * exp(s - m) with m a running row maximum that lags by less
+ * than a factor 2^4, so stored values are at most 256: the rounding error is
+ * at most 2^-4 of the value from 2^-6 up and at most 2^-10 below (the
+ * subnormal range).  O is accumulated in float32 and written as bf16.
  *
  * q [B, Hq, N, d], k and v [B, Hkv, N, d]: E4M3 codes, contiguous, 16-byte
  * aligned; o [B, Hq, N, d] bf16 and lse [B, Hq, N] float32 written by the
