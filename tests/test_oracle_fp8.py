@@ -239,3 +239,25 @@ def test_fp8_forward_rows_matches_full():
     orow, lrow = OF.fp8_forward_rows(q8[0, 0], k8[0, 0], v8[0, 0], 0.01, 0.02, 0.5, 0.2, True, rows)
     assert np.allclose(orow, o[0, 0, rows], rtol=1e-12, atol=1e-14)
     assert np.allclose(lrow, L[0, 0, rows], atol=1e-12)
+
+
+def test_draw_fp8_inputs():
+    """The seeded E4M3 inputs: no NaN codes, factors exact in float32, the
+    dequantised tensor within e4m3 rounding of the float32 draw, and the same
+    bits on every call."""
+    import attn_inputs
+    x = attn_inputs.draw_fp8(1, 2, 1, 64, 128, seed=11)
+    y = attn_inputs.draw_fp8(1, 2, 1, 64, 128, seed=11)
+    raw = attn_inputs.draw(1, 2, 1, 64, 64, 128, 11, torch.float32)
+    for n in ("q", "k", "v"):
+        codes = x[n].numpy()
+        assert codes.dtype == np.uint8
+        assert not np.any((codes & 0x7F) == 0x7F)
+        ds = x["descale_" + n]
+        assert float(np.float32(ds)) == ds
+        deq = OF.e4m3_decode(codes) * ds
+        ref = raw[n].double().numpy()
+        # round to nearest at 3 mantissa bits: relative 2^-4 for normals, 2^-10 * ds below 2^-6 * ds
+        assert np.all(np.abs(deq - ref) <= np.maximum(2.0 ** -4 * np.abs(ref), 2.0 ** -10 * ds) * (1 + 1e-6))
+        assert np.isclose(np.abs(deq).max(), 448 * ds, rtol=2.0 ** -4)
+        assert np.array_equal(codes, y[n].numpy()) and ds == y["descale_" + n]
