@@ -50,3 +50,36 @@ def test_two_rank_max_and_whole_job_value():
 def test_single_rank_is_identity():
     assert bench.max_over_ranks([3.0, 4.0]) == [3.0, 4.0]
     assert bench.whole_job_tflops(1, 2e12, 1000.0) == pytest.approx(2.0)
+
+
+def _run_reference(extra_env, workload="two_batch_bf16_n1024_d64"):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **extra_env)
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--steps", "3", "--warmup", "3", "--cpu-seconds", "0.3",
+                        "--workload", workload], capture_output=True, text=True, env=env,
+                       timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_line():
+    """The oracle arm prints one line with the base contract's keys, its own
+    workload's metric, and an e2e block with no host transfers."""
+    import attn_inputs
+    (out,) = _run_reference({"RANK": "0", "WORLD_SIZE": "1"})
+    w = attn_inputs.BY_NAME["two_batch_bf16_n1024_d64"]
+    assert out["impl"] == "reference" and out["metric"] == bench.metric_for(w)
+    assert out["value"] > 0 and out["unit"] == "TFLOP/s" and out["steps"] == 3
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["value"] == out["value"]
+    assert out["e2e"] == {"value": out["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
+    assert out["config"]["workload"] == "two_batch_bf16_n1024_d64"
+
+
+def test_reference_arm_other_ranks_are_silent():
+    assert _run_reference({"RANK": "1", "WORLD_SIZE": "2"}) == []
