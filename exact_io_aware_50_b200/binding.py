@@ -183,6 +183,49 @@ def _check(status, where):
         raise FaError(status, where)
 
 
+# Argument checks of the wrappers: shapes and dtypes first, then device and
+# layout; each raises ValueError before the library is called.
+def _check_qkv(where, q, k, v, dtypes):
+    """q [B, Hq, Nq, d]; k, v [B, Hkv, Nk, d]; one dtype among `dtypes`."""
+    if q.dim() != 4 or k.dim() != 4 or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"{where}: q must be [B, Hq, Nq, d] and k, v both [B, Hkv, Nk, d]")
+    if q.shape[0] != k.shape[0] or q.shape[3] != k.shape[3]:
+        raise ValueError(f"{where}: q and k disagree on B or d")
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in dtypes:
+        raise ValueError(f"{where}: q, k, v must share one dtype among {tuple(map(str, dtypes))}")
+
+
+def _check_bwd_in(where, q, o, lse, dout):
+    """o and dout shaped and typed like q; lse float32 [B, Hq, Nq]."""
+    import torch
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError(f"{where}: o and dout must have q's shape")
+    if o.dtype != q.dtype or dout.dtype != q.dtype:
+        raise ValueError(f"{where}: o and dout must have q's dtype")
+    if tuple(lse.shape) != tuple(q.shape[:3]) or lse.dtype != torch.float32:
+        raise ValueError(f"{where}: lse must be float32 [B, Hq, Nq]")
+
+
+def _check_cuda(where, *tensors):
+    for t in tensors:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{where}: inputs must be contiguous CUDA tensors")
+
+
+def _workspace(where, workspace, B, Hq, Nq, d, device):
+    """The caller's backward workspace, checked against fa_bwd_workspace_size
+    (the C entry points take a bare pointer and cannot), or a new one."""
+    import torch
+    need = fa_bwd_workspace_size(B, Hq, Nq, d)
+    if workspace is None:
+        return torch.empty(need, device=device, dtype=torch.uint8)
+    if (not workspace.is_cuda or not workspace.is_contiguous()
+            or workspace.numel() * workspace.element_size() < need):
+        raise ValueError(f"{where}: workspace must be a contiguous CUDA buffer of at least "
+                         f"{need} bytes")
+    return workspace
+
+
 def _shape(q, k):
     B, Hq, Nq, d = q.shape
     Bk, Hkv, Nk, dk = k.shape
@@ -200,16 +243,17 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
     """O, L = attention(q, k, v) for contiguous CUDA tensors [B, H, N, d]
     (bf16 -> fa_fwd, float32 -> fa_fwd_f32)."""
     import torch
+    _check_qkv("forward", q, k, v, (torch.bfloat16, torch.float32))
+    _check_cuda("forward", q, k, v)
     B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
     scale = d ** -0.5 if scale is None else float(scale)
-    for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("inputs must be contiguous CUDA tensors")
     o = torch.empty_like(q) if out is None else out
     L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32) if lse is None else lse
+    if (tuple(o.shape) != tuple(q.shape) or o.dtype != q.dtype or tuple(L.shape) != (B, Hq, Nq)
+            or L.dtype != torch.float32):
+        raise ValueError("forward: out must be shaped and typed like q, lse float32 [B, Hq, Nq]")
+    _check_cuda("forward", o, L)
     fn = fa_fwd if q.dtype == torch.bfloat16 else fa_fwd_f32
-    if q.dtype not in (torch.bfloat16, torch.float32):
-        raise ValueError("dtype must be bfloat16 or float32")
     _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), B, Hq, Hkv,
               Nq, Nk, d, scale, causal, _stream(q)), fn.__name__)
     return o, L
@@ -221,18 +265,21 @@ def forward_splitkv(q, k, v, scale=None, causal=False, num_splits=None, workspac
     Causal is bottom-right aligned (Nq <= Nk).  num_splits=None picks
     fa_fwd_splitkv_num_splits."""
     import torch
+    _check_qkv("forward_splitkv", q, k, v, (torch.bfloat16,))
+    _check_cuda("forward_splitkv", q, k, v)
     B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
     scale = d ** -0.5 if scale is None else float(scale)
-    for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
-            raise ValueError("inputs must be contiguous bfloat16 CUDA tensors")
     if num_splits is None:
         num_splits = fa_fwd_splitkv_num_splits(B, Hq, Nq, Nk, d)
     o = torch.empty_like(q)
     L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
+    need = max(fa_fwd_splitkv_workspace_size(B, Hq, Nq, d, num_splits), 1)
     if workspace is None:
-        workspace = torch.empty(max(fa_fwd_splitkv_workspace_size(B, Hq, Nq, d, num_splits), 1),
-                                device=q.device, dtype=torch.uint8)
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    elif (not workspace.is_cuda or not workspace.is_contiguous()
+          or workspace.numel() * workspace.element_size() < need):
+        raise ValueError(f"forward_splitkv: workspace must be a contiguous CUDA buffer of at "
+                         f"least {need} bytes")
     _check(fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
                           workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits,
                           _stream(q)), "fa_fwd_splitkv")
@@ -244,13 +291,12 @@ def forward_fp8(q, k, v, descale_q, descale_k, descale_v, scale=None, causal=Fal
     tensors of dtype float8_e4m3fn or uint8 (the codes); descale_*: the
     per-tensor dequantisation factors."""
     import torch
+    _check_qkv("forward_fp8", q, k, v, (torch.float8_e4m3fn, torch.uint8))
     B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
     if Nq != Nk:
-        raise ValueError("fa_fwd_fp8 takes Nq == Nk")
+        raise ValueError("forward_fp8: Nq must equal Nk")
+    _check_cuda("forward_fp8", q, k, v)
     scale = d ** -0.5 if scale is None else float(scale)
-    for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype not in (torch.float8_e4m3fn, torch.uint8):
-            raise ValueError("inputs must be contiguous float8_e4m3fn (or uint8) CUDA tensors")
     o = torch.empty(q.shape, device=q.device, dtype=torch.bfloat16)
     L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
     _check(fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
@@ -262,11 +308,10 @@ def forward_fp8(q, k, v, descale_q, descale_k, descale_v, scale=None, causal=Fal
 def forward_dropout(q, k, v, p_drop, seed, offset=0, scale=None, causal=False):
     """O, L with dropout on P (bf16, fa_fwd_dropout)."""
     import torch
+    _check_qkv("forward_dropout", q, k, v, (torch.bfloat16,))
+    _check_cuda("forward_dropout", q, k, v)
     B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
     scale = d ** -0.5 if scale is None else float(scale)
-    for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
-            raise ValueError("inputs must be contiguous bfloat16 CUDA tensors")
     o = torch.empty_like(q)
     L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
     _check(fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
@@ -279,12 +324,13 @@ def backward_dropout(q, k, v, o, lse, dout, p_drop, seed, offset=0, scale=None, 
                      workspace=None):
     """dQ, dK, dV of forward_dropout with the same seed and offset."""
     import torch
+    _check_qkv("backward_dropout", q, k, v, (torch.bfloat16,))
+    _check_bwd_in("backward_dropout", q, o, lse, dout)
+    _check_cuda("backward_dropout", q, k, v, o, lse, dout)
     B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
     scale = d ** -0.5 if scale is None else float(scale)
+    workspace = _workspace("backward_dropout", workspace, B, Hq, Nq, d, q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    if workspace is None:
-        workspace = torch.empty(fa_bwd_workspace_size(B, Hq, Nq, d), device=q.device,
-                                dtype=torch.uint8)
     _check(fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                           dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                           workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, p_drop, seed,
@@ -295,15 +341,13 @@ def backward_dropout(q, k, v, o, lse, dout, p_drop, seed, offset=0, scale=None, 
 def backward(q, k, v, o, lse, dout, scale=None, causal=False, workspace=None):
     """dQ, dK, dV for f = sum(O * dout); o and lse from ``forward``."""
     import torch
+    _check_qkv("backward", q, k, v, (torch.bfloat16, torch.float32))
+    _check_bwd_in("backward", q, o, lse, dout)
+    _check_cuda("backward", q, k, v, o, lse, dout)
     B, Hq, Hkv, Nq, Nk, d = _shape(q, k)
     scale = d ** -0.5 if scale is None else float(scale)
-    for t in (q, k, v, o, lse, dout):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("inputs must be contiguous CUDA tensors")
+    workspace = _workspace("backward", workspace, B, Hq, Nq, d, q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    if workspace is None:
-        workspace = torch.empty(fa_bwd_workspace_size(B, Hq, Nq, d), device=q.device,
-                                dtype=torch.uint8)
     fn = fa_bwd if q.dtype == torch.bfloat16 else fa_bwd_f32
     _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
               dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),

@@ -185,3 +185,41 @@ def test_size_limits():
     assert f(*(FAKE,) * 5, 1, 1, 1, 8, big_n, 64, 0.125, 0) == F.FA_ERR_UNSUPPORTED
     # B*Hq*Nq*d above 4e12 elements
     assert f(*(FAKE,) * 5, 4096, 1024, 1024, 8192, 8, 128, 0.125, 0) == F.FA_ERR_UNSUPPORTED
+
+
+def test_wrappers_reject_bad_tensors_before_the_library():
+    """The Python wrappers check shapes, dtypes, devices and the workspace size
+    and raise ValueError; nothing reaches the C entry points (CPU tensors)."""
+    import torch
+    bf = torch.bfloat16
+    q = torch.zeros(1, 2, 8, 64, dtype=bf)
+    k = torch.zeros(1, 1, 8, 64, dtype=bf)
+    with pytest.raises(ValueError, match="k, v both"):
+        F.forward(q, k, torch.zeros(1, 1, 9, 64, dtype=bf))
+    with pytest.raises(ValueError, match="disagree on B or d"):
+        F.forward(q, torch.zeros(1, 1, 8, 32, dtype=bf), torch.zeros(1, 1, 8, 32, dtype=bf))
+    with pytest.raises(ValueError, match="share one dtype"):
+        F.forward(q, k, k.float())
+    with pytest.raises(ValueError, match="share one dtype"):
+        F.forward(q.half(), k.half(), k.half())
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        F.forward(q, k, k)
+    with pytest.raises(ValueError, match="share one dtype"):
+        F.forward_fp8(q, k, k, 1.0, 1.0, 1.0)
+    q8 = torch.zeros(1, 2, 8, 128, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="Nq must equal Nk"):
+        F.forward_fp8(q8, torch.zeros(1, 1, 16, 128, dtype=torch.uint8),
+                      torch.zeros(1, 1, 16, 128, dtype=torch.uint8), 1.0, 1.0, 1.0)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        F.forward_fp8(q8, q8[:, :1].contiguous(), q8[:, :1].contiguous(), 1.0, 1.0, 1.0)
+    lse = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError, match="o and dout must have q's shape"):
+        F.backward(q, k, k, q[:, :1], lse, q)
+    with pytest.raises(ValueError, match="o and dout must have q's dtype"):
+        F.backward(q, k, k, q.float(), lse, q)
+    with pytest.raises(ValueError, match="lse must be float32"):
+        F.backward(q, k, k, q, lse.double(), q)
+    with pytest.raises(ValueError, match="lse must be float32"):
+        F.backward_dropout(q, k, k, q, lse[:, :, :4], q, 0.1, 1)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        F.backward(q, k, k, q, lse, q)
