@@ -25,6 +25,11 @@ int main(void) {
   printf("%d\n", fa_fwd(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 8, 8, 64, 0.125f, 0, NULL));
   printf("%d\n", fa_fwd_dropout(buf, buf, buf, buf, (float *)buf, 1, 1, 1, 8, 8, 64, 0.125f, 0,
                                 1.5f, 1ULL, 0ULL, (fa_stream_t)0));
+  /* e4m3 forward: a zero dequantisation factor, then an unsupported head dim */
+  printf("%d\n", fa_fwd_fp8(buf, buf, buf, buf, (float *)buf, 1, 1, 1, 8, 128, 0.125f, 0.0f,
+                            1.0f, 1.0f, 0, (fa_stream_t)0));
+  printf("%d\n", fa_fwd_fp8(buf, buf, buf, buf, (float *)buf, 1, 1, 1, 8, 64, 0.125f, 1.0f,
+                            1.0f, 1.0f, 0, (fa_stream_t)0));
   return 0;
 }
 """
@@ -47,3 +52,5 @@ def test_header_is_c_and_library_links(tmp_path):
     assert int(out[3]) == 9
     assert int(out[4]) == F.FA_ERR_INVALID_ARG
     assert int(out[5]) == F.FA_ERR_INVALID_ARG      # p_drop outside [0, 1)
+    assert int(out[6]) == F.FA_ERR_INVALID_ARG      # descale_q = 0
+    assert int(out[7]) == F.FA_ERR_UNSUPPORTED      # e4m3 at d = 64
