@@ -206,10 +206,23 @@ def _check_bwd_in(where, q, o, lse, dout):
         raise ValueError(f"{where}: lse must be float32 [B, Hq, Nq]")
 
 
-def _check_cuda(where, *tensors):
-    for t in tensors:
+def _check_cuda(where, q, *others):
+    """q and every other tensor: contiguous, on CUDA, and on q's device.  The
+    library launches on the current device, which the wrappers set to q's
+    (``_on``), so a tensor on another GPU would be read by kernels running on
+    the wrong one."""
+    for t in (q,) + others:
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{where}: inputs must be contiguous CUDA tensors")
+        if t.device != q.device:
+            raise ValueError(f"{where}: every tensor must be on q's device ({q.device}); "
+                             f"got one on {t.device}")
+
+
+def _on(q):
+    """Context that makes q's device current for one library call."""
+    import torch
+    return torch.cuda.device(q.device)
 
 
 def _workspace(where, workspace, B, Hq, Nq, d, device):
@@ -223,6 +236,9 @@ def _workspace(where, workspace, B, Hq, Nq, d, device):
             or workspace.numel() * workspace.element_size() < need):
         raise ValueError(f"{where}: workspace must be a contiguous CUDA buffer of at least "
                          f"{need} bytes")
+    if workspace.device != device:
+        raise ValueError(f"{where}: workspace must be on q's device ({device}); "
+                         f"got {workspace.device}")
     return workspace
 
 
@@ -252,10 +268,11 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
     if (tuple(o.shape) != tuple(q.shape) or o.dtype != q.dtype or tuple(L.shape) != (B, Hq, Nq)
             or L.dtype != torch.float32):
         raise ValueError("forward: out must be shaped and typed like q, lse float32 [B, Hq, Nq]")
-    _check_cuda("forward", o, L)
+    _check_cuda("forward", q, o, L)
     fn = fa_fwd if q.dtype == torch.bfloat16 else fa_fwd_f32
-    _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), B, Hq, Hkv,
-              Nq, Nk, d, scale, causal, _stream(q)), fn.__name__)
+    with _on(q):
+        _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), B, Hq, Hkv,
+                  Nq, Nk, d, scale, causal, _stream(q)), fn.__name__)
     return o, L
 
 
@@ -271,8 +288,6 @@ def forward_splitkv(q, k, v, scale=None, causal=False, num_splits=None, workspac
     scale = d ** -0.5 if scale is None else float(scale)
     if num_splits is None:
         num_splits = fa_fwd_splitkv_num_splits(B, Hq, Nq, Nk, d)
-    o = torch.empty_like(q)
-    L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
     need = max(fa_fwd_splitkv_workspace_size(B, Hq, Nq, d, num_splits), 1)
     if workspace is None:
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
@@ -280,9 +295,15 @@ def forward_splitkv(q, k, v, scale=None, causal=False, num_splits=None, workspac
           or workspace.numel() * workspace.element_size() < need):
         raise ValueError(f"forward_splitkv: workspace must be a contiguous CUDA buffer of at "
                          f"least {need} bytes")
-    _check(fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
-                          workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, num_splits,
-                          _stream(q)), "fa_fwd_splitkv")
+    elif workspace.device != q.device:
+        raise ValueError(f"forward_splitkv: workspace must be on q's device ({q.device}); "
+                         f"got {workspace.device}")
+    o = torch.empty_like(q)
+    L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
+    with _on(q):
+        _check(fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              L.data_ptr(), workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale,
+                              causal, num_splits, _stream(q)), "fa_fwd_splitkv")
     return o, L
 
 
@@ -299,9 +320,10 @@ def forward_fp8(q, k, v, descale_q, descale_k, descale_v, scale=None, causal=Fal
     scale = d ** -0.5 if scale is None else float(scale)
     o = torch.empty(q.shape, device=q.device, dtype=torch.bfloat16)
     L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
-    _check(fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
-                      B, Hq, Hkv, Nq, d, scale, descale_q, descale_k, descale_v, causal,
-                      _stream(q)), "fa_fwd_fp8")
+    with _on(q):
+        _check(fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
+                          B, Hq, Hkv, Nq, d, scale, descale_q, descale_k, descale_v, causal,
+                          _stream(q)), "fa_fwd_fp8")
     return o, L
 
 
@@ -314,9 +336,10 @@ def forward_dropout(q, k, v, p_drop, seed, offset=0, scale=None, causal=False):
     scale = d ** -0.5 if scale is None else float(scale)
     o = torch.empty_like(q)
     L = torch.empty(B, Hq, Nq, device=q.device, dtype=torch.float32)
-    _check(fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(),
-                          B, Hq, Hkv, Nq, Nk, d, scale, causal, p_drop, seed, offset, _stream(q)),
-           "fa_fwd_dropout")
+    with _on(q):
+        _check(fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              L.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, p_drop, seed,
+                              offset, _stream(q)), "fa_fwd_dropout")
     return o, L
 
 
@@ -331,10 +354,11 @@ def backward_dropout(q, k, v, o, lse, dout, p_drop, seed, offset=0, scale=None, 
     scale = d ** -0.5 if scale is None else float(scale)
     workspace = _workspace("backward_dropout", workspace, B, Hq, Nq, d, q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    _check(fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                          dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                          workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, p_drop, seed,
-                          offset, _stream(q)), "fa_bwd_dropout")
+    with _on(q):
+        _check(fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale,
+                              causal, p_drop, seed, offset, _stream(q)), "fa_bwd_dropout")
     return dq, dk, dv
 
 
@@ -349,7 +373,9 @@ def backward(q, k, v, o, lse, dout, scale=None, causal=False, workspace=None):
     workspace = _workspace("backward", workspace, B, Hq, Nq, d, q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     fn = fa_bwd if q.dtype == torch.bfloat16 else fa_bwd_f32
-    _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-              dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-              B, Hq, Hkv, Nq, Nk, d, scale, causal, _stream(q)), fn.__name__)
+    with _on(q):
+        _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                  dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                  workspace.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale, causal, _stream(q)),
+               fn.__name__)
     return dq, dk, dv

@@ -223,3 +223,74 @@ def test_wrappers_reject_bad_tensors_before_the_library():
         F.backward_dropout(q, k, k, q, lse[:, :, :4], q, 0.1, 1)
     with pytest.raises(ValueError, match="CUDA tensors"):
         F.backward(q, k, k, q, lse, q)
+
+
+class _FakeCuda:
+    """Stands in for a contiguous CUDA tensor on device `idx` without holding
+    memory; reaching the library through it fails the test."""
+
+    def __init__(self, shape, dtype, idx):
+        import torch
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+        self.device = torch.device("cuda", idx)
+        self.is_cuda = True
+
+    def dim(self):
+        return len(self.shape)
+
+    def is_contiguous(self):
+        return True
+
+    def numel(self):
+        n = 1
+        for s in self.shape:
+            n *= s
+        return n
+
+    def element_size(self):
+        import torch
+        return torch.empty(0, dtype=self.dtype).element_size()
+
+    def data_ptr(self):
+        raise AssertionError("a tensor on the wrong device reached the library")
+
+
+def test_wrappers_reject_tensors_on_another_device():
+    """Every tensor a wrapper passes (inputs, caller outputs, workspaces) must be
+    on q's device: the library launches on the current device, which the
+    wrappers make q's, so a tensor on another GPU is refused with ValueError
+    before anything is allocated or launched (stand-in tensors, no GPU)."""
+    import torch
+    bf = torch.bfloat16
+
+    def t(shape, idx, dtype=bf):
+        return _FakeCuda(shape, dtype, idx)
+
+    q0, k0, v0 = t((1, 2, 8, 64), 0), t((1, 1, 8, 64), 0), t((1, 1, 8, 64), 0)
+    lse0 = t((1, 2, 8), 0, torch.float32)
+    with pytest.raises(ValueError, match="q's device"):
+        F.forward(q0, t((1, 1, 8, 64), 1), v0)
+    with pytest.raises(ValueError, match="q's device"):
+        F.forward(q0, k0, t((1, 1, 8, 64), 1))
+    with pytest.raises(ValueError, match="q's device"):
+        F.forward(q0, k0, v0, out=t((1, 2, 8, 64), 1), lse=lse0)
+    with pytest.raises(ValueError, match="q's device"):
+        F.forward(q0, k0, v0, out=t((1, 2, 8, 64), 0), lse=t((1, 2, 8), 1, torch.float32))
+    with pytest.raises(ValueError, match="q's device"):
+        F.backward(q0, k0, v0, q0, lse0, t((1, 2, 8, 64), 1))
+    with pytest.raises(ValueError, match="q's device"):
+        F.backward(q0, k0, v0, t((1, 2, 8, 64), 1), lse0, q0)
+    ws1 = t((F.fa_bwd_workspace_size(1, 2, 8, 64),), 1, torch.uint8)
+    with pytest.raises(ValueError, match="workspace must be on q's device"):
+        F.backward(q0, k0, v0, q0, lse0, q0, workspace=ws1)
+    with pytest.raises(ValueError, match="workspace must be on q's device"):
+        F.backward_dropout(q0, k0, v0, q0, lse0, q0, 0.1, 1, workspace=ws1)
+    with pytest.raises(ValueError, match="q's device"):
+        F.forward_dropout(q0, k0, t((1, 1, 8, 64), 1), 0.1, 1)
+    with pytest.raises(ValueError, match="workspace must be on q's device"):
+        F.forward_splitkv(q0, k0, v0, num_splits=2, workspace=t((1 << 20,), 1, torch.uint8))
+    q8 = t((1, 2, 8, 128), 0, torch.uint8)
+    with pytest.raises(ValueError, match="q's device"):
+        F.forward_fp8(q8, t((1, 1, 8, 128), 1, torch.uint8), t((1, 1, 8, 128), 0, torch.uint8),
+                      1.0, 1.0, 1.0)
