@@ -8,15 +8,21 @@
 // plugins call cudaMalloc, or a latency-critical loop where cudaMalloc's
 // possible implicit device synchronisation is not acceptable.  For them this
 // file keeps the scratch in one fixed array in the library's device image,
-// sized kNoAllocScratchBytes.  Every GPU that loads the library reserves it
-// until the process exits.
+// sized kNoAllocScratchBytes.
 //
 // The first fa_bwd_noalloc call on a device looks up the array's device
-// address (cudaGetSymbolAddress, with that device current) and caches it;
-// make that first call before any stream capture.  All calls share the one
-// array and leave their contents in it: the kernels zero the dQ accumulator
-// and rewrite D on every call, and two calls whose kernels overlap on the GPU
-// (different streams, or different host threads on one device) race on it.
+// address (cudaGetSymbolAddress, with that device current) and caches it.
+// The runtime loads device code lazily, so that lookup is also what creates
+// the array on the device: the first call makes a 32 MiB allocation inside
+// the runtime, may synchronise the device and fails with FA_ERR_CUDA when the
+// memory is not there.  Make that first call during set-up, before any stream
+// capture; the array then stays on the device until the process exits.  The
+// cached address is that of the device's primary context and goes stale after
+// cudaDeviceReset (as does the error-word address of fa_capi.cu).  All calls
+// share the one array and leave their contents in it: the kernels zero the
+// dQ accumulator and rewrite D on every call, and two calls whose kernels
+// overlap on the GPU (different streams, or different host threads on one
+// device) race on it.
 #include <atomic>
 
 #include "../../include/fa.h"

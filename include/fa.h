@@ -226,15 +226,23 @@ int fa_bwd_f32(const float *q, const float *k, const float *v, const float *o,
  * that owns the device memory pool, or a loop that must not risk the device
  * synchronisation cudaMalloc can cause).  Same arguments and results as
  * fa_bwd, minus the workspace: the scratch lives in one fixed 32 MiB array
- * inside the library (reserved on every GPU that loads it, until exit).
- * The FlashAttention pages describe no such call; it is an interface convenience.
+ * inside the library, held on each GPU from the first call there until the
+ * process exits.  The FlashAttention pages describe no such call; it is an
+ * interface convenience.
  * Returns FA_ERR_UNSUPPORTED, without touching the device, when the problem
  * needs more scratch than that (about 4*B*Hq*(Nq*(d+2) + d) bytes plus
- * padding, e.g. more than about 64,000 query rows B*Hq*Nq at d = 128).  The first call on a
- * device looks up the array's address, so make it before any stream capture.
+ * padding, e.g. more than about 64,000 query rows B*Hq*Nq at d = 128).
+ * First call on a device: the CUDA runtime loads the library's device code
+ * lazily, so the array is created then (a 32 MiB device allocation made by
+ * the runtime, which can synchronise the device and can fail with FA_ERR_CUDA
+ * when the device is out of memory) and its address is looked up and cached.
+ * Make that first call during set-up, before any stream capture; later calls
+ * allocate nothing and do not synchronise.  The cached address belongs to the
+ * device's primary context: after cudaDeviceReset the library must be
+ * reloaded (the same holds for the device error word of every entry point).
  * Every call uses the same array: calls whose kernels overlap on the GPU
  * (other streams or threads on the same device) race and must be ordered by
- * the caller.  Allocates nothing.
+ * the caller.
  */
 int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
                    const float *lse, const void *dout, void *dq, void *dk, void *dv,
