@@ -34,8 +34,8 @@ import numpy as np
 
 from .attention import forward
 
-__all__ = ["e4m3_decode", "fp8_forward", "fp8_forward_rows", "p_quantisation_bounds",
-           "P_SHIFT_LOG2", "P_RESCALE_LOG2"]
+__all__ = ["e4m3_decode", "e4m3_round", "fp8_forward", "fp8_forward_rows",
+           "p_quantisation_bounds", "stored_p_forward", "P_SHIFT_LOG2", "P_RESCALE_LOG2"]
 
 # Reading of the kernel's P storage, fixed by the method's FP8 variant here:
 # p is stored as e4m3(2^P_SHIFT_LOG2 * 2^(x - m_run)) where m_run (base-2
@@ -114,3 +114,55 @@ def p_quantisation_bounds(q2, k2, v2, scale, causal, rows=None):
     kappa = np.where(w > 0, kappa, 0.0)
     rms = float(np.sqrt(np.sum((kappa ** 2) @ (v2 ** 2))))
     return elementwise, rms
+
+
+def e4m3_round(y) -> np.ndarray:
+    """Round non-negative float64 values to the nearest OCP E4M3 value, ties
+    to even, saturating at the largest finite value 448 (the satfinite
+    conversion).  Subnormals: multiples of 2^-9 below 2^-6; normals: 3
+    mantissa bits, a step of 2^(e-3) in [2^e, 2^(e+1))."""
+    y = np.asarray(y, dtype=np.float64)
+    if np.any(y < 0) or np.any(np.isnan(y)):
+        raise ValueError("e4m3_round takes non-negative values")
+    out = np.empty_like(y)
+    sub = y < 2.0 ** -6
+    out[sub] = np.rint(y[sub] / 2.0 ** -9) * 2.0 ** -9
+    nz = ~sub
+    e = np.floor(np.log2(np.where(nz, y, 1.0)))
+    step = np.exp2(e - 3)
+    out[nz] = (np.rint(y / step) * step)[nz]
+    return np.minimum(out, 448.0)
+
+
+def stored_p_forward(x2, v2, shift=P_SHIFT_LOG2, tau=P_RESCALE_LOG2, block=128, group=32):
+    """O of one head when P is held as the kernel's reading above holds it:
+    the online softmax with deferred normalisation (blog section 4.1) in
+    float64 over key blocks of `block`, each stored value rounded by
+    ``e4m3_round``: y = e4m3(2^shift 2^(x - m)), the row sum over the
+    unrounded values, and the running maximum m (base 2) refreshed only when
+    some row of a `group` of consecutive rows grows by more than `tau` (the
+    first block always sets it).  x2: scaled scores in base 2, [n, nk], -inf
+    where masked; v2: [nk, d] float64.  This models the error source that
+    ``p_quantisation_bounds`` bounds; it is not the definition of O."""
+    x2 = np.asarray(x2, dtype=np.float64)
+    v2 = np.asarray(v2, dtype=np.float64)
+    n, nk = x2.shape
+    m = np.full(n, -np.inf)
+    l = np.zeros(n)
+    acc = np.zeros((n, v2.shape[1]))
+    for j0 in range(0, nk, block):
+        x = x2[:, j0:j0 + block]
+        m_new = np.maximum(m, x.max(axis=1))
+        for g0 in range(0, n, group):
+            sl = slice(g0, g0 + group)
+            if j0 == 0 or np.any(m_new[sl] - m[sl] > tau):
+                alpha = np.where(np.isfinite(m[sl]), np.exp2(m[sl] - m_new[sl]), 0.0)
+                acc[sl] *= alpha[:, None]
+                l[sl] *= alpha
+                m[sl] = m_new[sl]
+        mu = np.where(np.isfinite(m), m, 0.0)
+        y = np.exp2(x - mu[:, None] + shift)
+        l += y.sum(axis=1)
+        acc += e4m3_round(y) @ v2[j0:j0 + block]
+    return acc / l[:, None]
+

@@ -123,3 +123,62 @@ def test_fp8_descale_fold():
     z["descale_q"] = 2.0 * x["descale_q"]
     o3, l3 = _run(z, True, 0.05)
     assert np.array_equal(o3, o1) and np.array_equal(l3, l1)
+
+
+def _e4m3_code(x):
+    """Code of an exactly representable E4M3 value."""
+    c = torch.tensor([x], dtype=torch.float64).to(torch.float8_e4m3fn).view(torch.uint8).item()
+    assert OF.e4m3_decode(np.array([c], np.uint8))[0] == x, x
+    return c
+
+
+def test_fp8_p_storage_matches_the_bound_model():
+    """The kernel's P storage is what oracle.fp8's error model assumes:
+    e4m3(2^P_SHIFT_LOG2 2^(x - m)) with a running maximum that lags by at most
+    P_RESCALE_LOG2.  Every query row is q = (1, 1/2, 0, ...) and each key's
+    first two components set its score (scale = ln 2, so scores are in base
+    2); probe keys sit where the stored value lands clearly on or off the
+    e4m3 subnormal grid, next to block maxima that grow by exactly 4 and then
+    by 9.  The kernel's O must equal stored_p_forward's within one bf16 ulp,
+    and the model with shift 3 or 5, or threshold 3 or 9, must give an O that
+    differs by many ulps, so a change on either side fails this test."""
+    N, d = 384, 128
+    # base-2 scores, value columns: (key, score, column of its value 256, or
+    # column 0 with value 1 for the block maxima)
+    probes = [(0, 0.0, 0), (1, -13.5, 1), (2, -13.0, 2),        # block 0, max 0
+              (128, 4.0, 0), (129, -10.5, 3),                   # block 1, max grows by 4
+              (256, 9.0, 0), (257, -4.5, 4)]                    # block 2, max grows by 9
+    a = np.full(N, -448.0)
+    vcol = {}
+    for key, score, col in probes:
+        a[key] = score
+        vcol[key] = col
+    k = np.zeros((N, d))
+    k[:, 0] = np.ceil(a)                 # representable integers for these scores
+    k[:, 1] = 2.0 * (a - np.ceil(a))     # 0 or -1, so that a = k0 + k1 / 2
+    v = np.zeros((N, d))
+    for key, col in vcol.items():
+        v[key, col] = 1.0 if col == 0 else 256.0
+    q = np.zeros((N, d))
+    q[:, 0], q[:, 1] = 1.0, 0.5
+    assert np.array_equal(q @ k.T, np.tile(a, (N, 1)))
+    enc = np.vectorize(_e4m3_code)
+    codes = {n: torch.from_numpy(enc(t).astype(np.uint8)).reshape(1, 1, N, d)
+             for n, t in (("q", q), ("k", k), ("v", v))}
+    scale = float(np.float32(np.log(2.0)))
+    o, lse = F.forward_fp8(codes["q"].cuda(), codes["k"].cuda(), codes["v"].cuda(), 1.0, 1.0, 1.0,
+                           scale=scale, causal=False)
+    torch.cuda.synchronize()
+    assert F.fa_device_status() == F.FA_OK
+    o = f64(o)[0, 0]
+    x2 = np.tile(a, (N, 1))
+
+    def model(shift, tau):
+        return OF.stored_p_forward(x2, v, shift=shift, tau=tau)
+
+    ref = model(OF.P_SHIFT_LOG2, OF.P_RESCALE_LOG2)
+    ulp = 2.0 * half_ulp_bf16(ref)
+    assert np.all(np.abs(o - ref) <= ulp), np.max(np.abs(o - ref) / ulp)
+    for shift, tau in ((3, 4), (5, 4), (4, 3), (4, 9)):
+        alt = model(shift, tau)
+        assert np.max(np.abs(alt - ref) / ulp) > 8, (shift, tau)

@@ -261,3 +261,45 @@ def test_draw_fp8_inputs():
         assert np.all(np.abs(deq - ref) <= np.maximum(2.0 ** -4 * np.abs(ref), 2.0 ** -10 * ds) * (1 + 1e-6))
         assert np.isclose(np.abs(deq).max(), 448 * ds, rtol=2.0 ** -4)
         assert np.array_equal(codes, y[n].numpy()) and ds == y["descale_" + n]
+
+
+# ------------------------------------------- stored-P model of the kernel
+def test_e4m3_round_grid_midpoints_and_saturation():
+    """e4m3_round: every finite non-negative E4M3 value is a fixed point;
+    midpoints between neighbours round as torch's float8_e4m3fn conversion
+    (round to nearest even); values above 448 saturate (satfinite)."""
+    vals = OF.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    assert np.array_equal(OF.e4m3_round(vals), vals)
+    mid = (vals[1:] + vals[:-1]) / 2
+    assert np.array_equal(OF.e4m3_round(mid), _e4m3_round(mid))
+    r = RNG.uniform(0, 448, 20000) * np.exp2(RNG.integers(-14, 1, 20000))
+    assert np.array_equal(OF.e4m3_round(r), _e4m3_round(r))
+    assert np.all(OF.e4m3_round(np.array([448.0, 460.0, 480.0, 1e9])) == 448.0)
+
+
+def test_stored_p_forward_matches_simulation_with_library_rounding():
+    """stored_p_forward equals quantised_online above (scores from the
+    oracle's definition, rounding by torch's e4m3 conversion)."""
+    n, d = 300, 64
+    q = RNG.standard_normal((n, d)) * 3.0
+    k = RNG.standard_normal((n, d))
+    v = RNG.standard_normal((n, d))
+    scale = d ** -0.5
+    for causal in (False, True):
+        x2 = OA.scores(q, k, scale, causal) / np.log(2.0)
+        a = OF.stored_p_forward(x2, v)
+        b = quantised_online(q, k, v, scale, causal)
+        assert np.max(np.abs(a - b)) <= 1e-12
+
+
+def test_stored_p_forward_is_exact_on_the_grid():
+    """When every stored value lands on the e4m3 grid (integer base-2 scores
+    close to the row maximum), the model reproduces softmax(x) V exactly,
+    whichever running maximum it used: a closed form for its recurrence."""
+    n, nk, d = 64, 384, 16
+    x2 = RNG.integers(-9 - OF.P_SHIFT_LOG2, 1, (n, nk)).astype(np.float64)
+    x2[:, 200] += 4      # a growth of exactly tau: no rescale, stored 2^8
+    v = RNG.standard_normal((nk, d))
+    w = np.exp2(x2 - x2.max(axis=1, keepdims=True))
+    exact = (w / w.sum(axis=1, keepdims=True)) @ v
+    assert np.max(np.abs(OF.stored_p_forward(x2, v) - exact)) <= 1e-12
