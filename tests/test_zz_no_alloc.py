@@ -35,7 +35,8 @@ def test_noalloc_refuses_problems_larger_than_its_scratch():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("shape", [(1, 4, 2, 1000, 128, True), (2, 2, 2, 700, 64, False)])
+@pytest.mark.parametrize("shape", [(1, 4, 2, 1000, 128, True), (2, 2, 2, 700, 64, False),
+                                   (1, 2, 2, 512, 256, True)])
 def test_noalloc_matches_workspace_backward_twice(shape):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
