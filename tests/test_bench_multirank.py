@@ -79,6 +79,14 @@ def test_reference_arm_line():
     assert out["e2e"] == {"value": out["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                           "d2h_bytes_per_step": 0}
     assert out["config"]["workload"] == "two_batch_bf16_n1024_d64"
+    # the same configuration dict as the GPU arm prints for this workload
+    assert out["config"] == bench.config_dict(w, 1)
+    # the step time is extrapolated from the units the oracle did run, and says so
+    assert out["extrapolated"] is True
+    m = out["measured"]
+    assert m["units_timed"] >= 1 and m["seconds"] > 0 and m["units_per_step"] == w.B * w.Hq
+    assert abs(out["ms_per_step"] - m["ms_per_unit"] * m["units_per_step"]) <= \
+        0.5 * out["ms_per_step"] + 1.0
 
 
 def test_reference_arm_other_ranks_are_silent():
