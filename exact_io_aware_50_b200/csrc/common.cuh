@@ -144,6 +144,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint
       : "memory");
 }
 
+// Bring a 3-D tile into L2 ahead of its load (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void *tmap, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
 // Non-tensor bulk reduce-add of float32 from shared to global memory.
 __device__ __forceinline__ void bulk_reduce_add_f32(float *gdst, uint32_t src, uint32_t bytes) {
   asm volatile(

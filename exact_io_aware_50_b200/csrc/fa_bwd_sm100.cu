@@ -22,7 +22,7 @@
 //   prep   1. c per (batch, key/value head) into the workspace;
 //          2. per query row: D_i, L2_i = log2e * L_i - scale * log2e * q_i . c,
 //             padded to 128-row blocks, and the zeroed f32 dQ accumulator;
-//   dkdv   one CTA per (batch, key/value head, 128-row key block); K - c and
+//   dkdv   work unit = (batch, key/value head, 128-row key block); K - c and
 //          V stay in shared memory and dK, dV in TMEM for the whole loop over
 //          the query heads of the group and their query blocks, so dK and dV
 //          need no atomics.  Per step (key rows on the 128 TMEM lanes):
@@ -34,8 +34,9 @@
 //          and readout warps add dQ_i^T into the f32 accumulator with float32
 //          reductions.  Q_i, dO_i and the row vectors L2_i, D_i arrive
 //          through a ring of TMA copies.
-//          d = 64, 128: bwd_wide_kernel, 128-row query blocks, one TMEM score
-//          set and a two-phase elementwise stage (see its comment block).
+//          d = 64, 128: bwd_wide_kernel, persistent (one CTA per SM taking
+//          units from a counter), 128-row query blocks, one TMEM score set and
+//          a two-phase elementwise stage (see its comment block).
 //          d = 256: the dK and dV accumulators alone fill TMEM, so
 //          bwd_kernel runs two passes over the same key blocks, dV (S^T,
 //          P^T, dV) then dK and dQ, with 64-row query blocks and two TMEM
@@ -48,6 +49,13 @@
 
 #include "common.cuh"
 #include "launch.h"
+
+#ifndef BWD_PERSIST
+#define BWD_PERSIST 1
+#endif
+#ifndef BWD_GROUP_BYTES
+#define BWD_GROUP_BYTES 32e6
+#endif
 
 namespace fa {
 namespace {
@@ -142,8 +150,10 @@ struct BwdParams {
   const float *dsum;       // [B*Hq][Npad]
   const float *cvec;       // [B*Hkv][D]
   float *dq_acc;           // [B, Hq, Nq, D]
+  int *sched;              // persistent dK/dV kernel: units handed out so far (beyond the grid)
   __nv_bfloat16 *dk, *dv;  // [B, Hkv, Nk, D]
   int Hq, Hkv, Nq, Nk, npad, nqb, nkb, BHkv;
+  int hg;                  // key/value heads per group of the unit order
   float scale, scale_log2;
   int causal;
   // dropout on P (wide kernel, DROP instances): keep when the Philox word is
@@ -676,13 +686,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 // overlaps dV(i+1).  P^T is kept in registers between the phases in bf16, the
 // precision the dV MMA also uses.
 //
+// Two step orders (BwdWideCfg::EARLY_S):
+//   default  dV(i)  dK(i)  S^T(i+1)  dQ^T(i)  dP^T(i+1), dK's A operand (dS^T)
+//            from TMEM: S^T(i+1) waits for phase 2 of step i;
+//   EARLY_S  dV(i)  S^T(i+1)  dQ^T(i)  dK(i)  dP^T(i+1), dS^T only in shared
+//            memory (A operand of dK, K-major): S^T(i+1) is computed while
+//            phase 2 of step i runs, so phase 1 of step i+1 follows phase 2 at
+//            once.  Measured on B200 (dK/dV kernel, same build otherwise):
+//            d = 64 faster (causal B8 H16 N2048: 0.745 -> 0.684 ms), d = 128
+//            slower (causal B4 H16 N4096: 0.875 -> 0.952 ms): the extra shared-
+//            memory operand reads and the dQ reductions that then overlap the
+//            tensor-core work cost more than the shorter chain gains.
+// With EARLY_S, phase 2 writes dS^T(i) to shared memory only after dP^T(i)
+// has completed, which implies dQ^T(i-1) and dK(i-1), issued before it, are
+// done reading the previous dS^T.
+//
+// Persistent CTAs, one per SM.  CTA c starts with unit c of the list; the
+// producer takes the next unit from a counter in the workspace (atomicAdd;
+// the prep stage zeroes it) once it has issued all loads of its current unit,
+// so the SM that frees up first gets the heaviest unit left, and it hands the
+// unit to the other roles through a four-entry shared-memory queue.  The next
+// unit's K and V are prefetched into L2 at that point and loaded into shared
+// memory when the current unit's last MMA completes; its first Q/dO tiles are
+// already in the ring.  The epilogue reads dV and dK out of TMEM and releases
+// them (acc_empty) before storing, and the next unit's first dV/dK MMAs wait
+// for that release.  Units are listed in groups of key/value heads whose
+// f32 dQ accumulator, Q and dO take about 32 MB (the dQ reductions of a group
+// stay in L2), the key blocks with most query blocks first within a group
+// (causal).  Measured on B200 against one CTA per unit with the same steps:
+// causal B4 H16 N4096 d128 0.889 -> 0.854 ms, GQA B1 Hq32 Hkv8 N16384
+// 6.35 -> 6.12 ms, causal B64 H16 N512 d128 0.520 -> 0.453 ms.
+//
 // Warps: 0-7 elementwise (two warpgroups, 64 query columns each; warpgroup 0
-// writes dV and warpgroup 1 dK at the end), 8-15 dQ^T readout (two warps per
-// TMEM lane quarter, two 32-column chunks each, float32 reductions into the
-// accumulator), 16 TMA producer, 17 MMA issuer (both in lane 0).
-template <int D_, int QS_>
+// writes dV and warpgroup 1 dK at the end of a unit), 8-15 dQ^T readout (two
+// warps per TMEM lane quarter, two 32-column chunks each, float32 reductions
+// into the accumulator), 16 TMA producer, 17 MMA issuer (both in lane 0).
+// EARLY_S_: the step order that issues S^T(i+1) right after dV(i) and takes
+// dK's A operand (dS^T) from shared memory (see the comment block above).
+template <int D_, int QS_, bool EARLY_S_>
 struct BwdWideCfg {
   static constexpr int D = D_, QS = QS_;
+  static constexpr bool EARLY_S = EARLY_S_;
   static constexpr int BN = 128, BM = 128;
   static constexpr int DCH = D / 64;
   static constexpr int KV_CHUNK = BN * 128;
@@ -701,10 +745,10 @@ struct BwdWideCfg {
   static constexpr int OFF_DD = OFF_L2 + QS * ROWVEC;
   static constexpr int OFF_BAR = OFF_DD + QS * ROWVEC;
   // kv, kc, q_full[QS], q_empty[QS], s_full, dp_full, p_full, ds_full,
-  // dq_full, dq_empty, final, drain
-  static constexpr int NBAR = 2 + 2 * QS + 8;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16;
+  // dq_full, dq_empty, final, drain, acc_empty, unit_full[4], unit_empty[4]
+  static constexpr int NBAR = 2 + 2 * QS + 9 + 8;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;   // tmem slot, abort flag, unit queue[4]
+  static constexpr int SMEM = OFF_MISC + 32;
   static constexpr int TM_DV = 0, TM_DK = D, TM_A = 2 * D, TM_B = 2 * D + 128;
   static constexpr int TM_ALLOC = 512;
   static constexpr int THREADS = 18 * 32;
@@ -732,28 +776,51 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int B_KV = 0, B_KC = 1, B_QFULL = 2, B_QEMPTY = 2 + C::QS, B_SFULL = 2 + 2 * C::QS,
             B_DPFULL = B_SFULL + 1, B_PFULL = B_SFULL + 2, B_DSFULL = B_SFULL + 3,
             B_DQFULL = B_SFULL + 4, B_DQEMPTY = B_SFULL + 5, B_FINAL = B_SFULL + 6,
-            B_DRAIN = B_SFULL + 7;
+            B_DRAIN = B_SFULL + 7, B_ACCEMPTY = B_SFULL + 8, B_UFULL = B_SFULL + 9,
+            B_UEMPTY = B_UFULL + 4;
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
+  volatile int *s_queue = (volatile int *)(smem + C::OFF_MISC + 16);   // unit of the k-th turn, k % 4
   const float *s_l2 = (const float *)(smem + C::OFF_L2);
   const float *s_dd = (const float *)(smem + C::OFF_DD);
 
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
-
-  // Work unit: head by head (batch, key/value head), and inside a head the
-  // key blocks with the most query blocks first (causal).
-  const int unit = blockIdx.x;
-  const int jblk = unit % p.nkb;
-  const int bhkv = unit / p.nkb;
-  const int b = bhkv / p.Hkv, hkv = bhkv % p.Hkv;
   const int g = p.Hq / p.Hkv;
-  const int kv0 = jblk * C::BN;
-  const int i0 = p.causal ? kv0 / C::BM : 0;  // first query block that sees this key block
-  const int nq_eff = p.nqb - i0;
-  const int nsteps = nq_eff > 0 ? g * nq_eff : 0;
-  auto step_head = [&](int s) { return hkv * g + s / nq_eff; };
-  auto step_qblk = [&](int s) { return i0 + s % nq_eff; };
+
+  // Work units: (batch, key/value head, 128-row key block).  The unit list
+  // runs over groups of hg heads one after the other; inside a group the
+  // key blocks with the most query blocks come first (causal), heads
+  // interleaved.  Persistent CTAs (one per SM): CTA c starts with unit c;
+  // after that the producer takes the next unit of the list from a counter
+  // in the workspace (atomicAdd) when it has issued the loads of its current
+  // one, so the SM that frees up first gets the heaviest unit left (the order
+  // a hardware block scheduler would give, without a CTA's set-up and
+  // teardown between units).  The producer hands each unit to the other
+  // roles through a four-entry queue in shared memory (-1 ends the
+  // sequence); barrier phases follow the count of units (uc) and of steps
+  // (gs) this CTA has processed.
+  const int total_units = p.nkb * p.BHkv;
+  const int G = (int)gridDim.x;
+  struct Unit {
+    int bhkv, b, hkv, kv0, i0, nq_eff, nsteps;
+  };
+  auto decode = [&](int u) {
+    Unit U;
+    const int grp = u / (p.hg * p.nkb), wu = u % (p.hg * p.nkb);
+    const int hn = min(p.hg, p.BHkv - grp * p.hg);
+    const int jblk = wu / hn;
+    U.bhkv = grp * p.hg + wu % hn;
+    U.b = U.bhkv / p.Hkv;
+    U.hkv = U.bhkv % p.Hkv;
+    U.kv0 = jblk * C::BN;
+    U.i0 = p.causal ? U.kv0 / C::BM : 0;   // first query block that sees this key block
+    U.nq_eff = p.nqb - U.i0;
+    U.nsteps = U.nq_eff > 0 ? g * U.nq_eff : 0;
+    return U;
+  };
+  auto step_head = [&](const Unit &U, int s) { return U.hkv * g + s / U.nq_eff; };
+  auto step_qblk = [&](const Unit &U, int s) { return U.i0 + s % U.nq_eff; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_KV), 1);
@@ -770,6 +837,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(bar(B_DQEMPTY), 256);
     mbar_init(bar(B_FINAL), 1);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_ACCEMPTY), 256);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(bar(B_UFULL + s), 1);
+      mbar_init(bar(B_UEMPTY + s), 17);   // MMA issuer + 8 elementwise + 8 readout warps
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -794,19 +866,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (lane == 0) {
       int last_phase[C::QS];
       for (int s = 0; s < C::QS; ++s) last_phase[s] = -1;
+      int kv_phase = -1;
       bool ok = true;
-      mbar_arrive_expect_tx(bar(B_KV), 2 * C::KV_TILE);
-      for (int c = 0; c < C::DCH; ++c) {
-        tma_load_3d(sbase + C::OFF_K + c * C::KV_CHUNK, &tmK, bar(B_KV), c * 64, kv0, bhkv);
-        tma_load_3d(sbase + C::OFF_V + c * C::KV_CHUNK, &tmV, bar(B_KV), c * 64, kv0, bhkv);
-      }
-      for (int i = 0; i < nsteps && ok; ++i) {
-        const int st = i % C::QS;
-        const uint32_t ph = (i / C::QS) & 1;
-        ok = bounded_wait(bar(B_QEMPTY + st), ph ^ 1, wc);
-        if (!ok) break;
-        const int h = step_head(i), qb = step_qblk(i);
-        const int bh = b * p.Hq + h;
+      int uc = 0, gs = 0;
+      // Q_i, dO_i and the row slices of L2 and D of step i of unit U
+      auto load_step = [&](const Unit &U, int i) {
+        const int gi = gs + i;
+        const int st = gi % C::QS;
+        const uint32_t ph = (gi / C::QS) & 1;
+        if (!bounded_wait(bar(B_QEMPTY + st), ph ^ 1, wc)) return false;
+        const int h = step_head(U, i), qb = step_qblk(U, i);
+        const int bh = U.b * p.Hq + h;
         const size_t vrow = (size_t)bh * p.npad + (size_t)qb * C::BM;
         const uint32_t fb = bar(B_QFULL + st);
         mbar_arrive_expect_tx(fb, 2 * C::Q_TILE + 2 * C::ROWVEC);
@@ -819,9 +889,50 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         bulk_load(sbase + C::OFF_L2 + st * C::ROWVEC, p.l2 + vrow, C::ROWVEC, fb);
         bulk_load(sbase + C::OFF_DD + st * C::ROWVEC, p.dsum + vrow, C::ROWVEC, fb);
         last_phase[st] = ph;
+        return true;
+      };
+      int u = (int)blockIdx.x;
+      for (int k = 0; ok; ++k) {
+        // publish this turn's unit (or the end of the sequence)
+        ok = bounded_wait(bar(B_UEMPTY + (k & 3)), ((k >> 2) & 1) ^ 1, wc);
+        if (!ok) break;
+        s_queue[k & 3] = u < total_units ? u : -1;
+        mbar_arrive(bar(B_UFULL + (k & 3)));
+        if (u >= total_units) break;
+        const Unit U = decode(u);
+        if (U.nsteps == 0) {
+          u = G + atomicAdd(p.sched, 1);
+          continue;
+        }
+        // the first ring slots of this unit, then K and V once the previous
+        // unit's MMAs (the last readers of K and V) are done, then the rest
+        const int pre = min(C::QS, U.nsteps);
+        for (int i = 0; i < pre && ok; ++i) ok = load_step(U, i);
+        if (ok && uc > 0) ok = bounded_wait(bar(B_FINAL), (uc - 1) & 1, wc);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(B_KV), 2 * C::KV_TILE);
+        for (int c = 0; c < C::DCH; ++c) {
+          tma_load_3d(sbase + C::OFF_K + c * C::KV_CHUNK, &tmK, bar(B_KV), c * 64, U.kv0, U.bhkv);
+          tma_load_3d(sbase + C::OFF_V + c * C::KV_CHUNK, &tmV, bar(B_KV), c * 64, U.kv0, U.bhkv);
+        }
+        kv_phase = uc & 1;
+        for (int i = pre; i < U.nsteps && ok; ++i) ok = load_step(U, i);
+        gs += U.nsteps;
+        ++uc;
+        // the next unit, taken once this one's loads are all issued; its K
+        // and V tiles go to L2 now, so their load after this unit's last MMA
+        // does not wait on DRAM
+        u = G + atomicAdd(p.sched, 1);
+        if (u < total_units) {
+          const Unit N = decode(u);
+          for (int c = 0; c < C::DCH; ++c) {
+            tma_prefetch_l2_3d(&tmK, c * 64, N.kv0, N.bhkv);
+            tma_prefetch_l2_3d(&tmV, c * 64, N.kv0, N.bhkv);
+          }
+        }
       }
       if (!ok) {
-        (void)drain_wait(bar(B_KV), 0, p.err, kWaitLimitNs);
+        if (kv_phase >= 0) (void)drain_wait(bar(B_KV), kv_phase, p.err, kWaitLimitNs);
         for (int s = 0; s < C::QS; ++s)
           if (last_phase[s] >= 0) (void)drain_wait(bar(B_QFULL + s), last_phase[s], p.err, kWaitLimitNs);
       }
@@ -840,6 +951,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint64_t dO_km = sw128_desc(sbase + C::OFF_DO, 16, 1024);
     const uint64_t dO_mn = sw128_desc(sbase + C::OFF_DO, C::Q_CHUNK, 1024);
     const uint64_t dS_mn = sw128_desc(sbase + C::OFF_DS, C::DS_CHUNK, 1024);
+    const uint64_t dS_km = sw128_desc(sbase + C::OFF_DS, 16, 1024);
     // S^T = (K-c) Q^T (A region), dP^T = V dO^T (B region); K = d, 16 per MMA
     auto issue_SP = [&](uint64_t a0, uint64_t b0, int st, uint32_t dst) {
       const uint64_t bt = desc_add(b0, st * C::Q_TILE);
@@ -860,6 +972,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mma_ts(tmem + acc, tmem + C::TM_A + (kk >> 1) * 32 + (kk & 1) * 8 + col,
                desc_add(bt, kk * 2048), IDESC_KV, (!first) || kk > 0);
     };
+    // EARLY_S: dK += dS^T Q_i with dS^T read from shared memory (K-major: key
+    // rows of 64-query-column chunks), so A is free for S^T(i+1) once dV(i)
+    // has read P^T(i).
+    auto issue_dk_smem = [&](int st, bool first) {
+      const uint64_t bt = desc_add(dQ_mn, st * C::Q_TILE);
+#pragma unroll
+      for (int kk = 0; kk < C::BM / 16; ++kk)
+        mma_ss(tmem + C::TM_DK, desc_add(dS_km, (kk >> 2) * C::DS_CHUNK + (kk & 3) * 32),
+               desc_add(bt, kk * 2048), IDESC_KV, (!first) || kk > 0);
+    };
     // dQ^T = A^T dS^T, K = 128 key rows (16 per MMA), M = 128 rows of A^T:
     // (K-c)^T for d = 128, [(K-c)^T ; V^T] for d = 64 (the V half unused).
     auto issue_dq = [&]() {
@@ -869,50 +991,97 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                kk > 0);
     };
     if (lane == 0) {
-      bool ok = bounded_wait(bar(B_KC), 0, wc);   // K - c in place
-      if (ok && nsteps > 0) {
-        ok = bounded_wait(bar(B_QFULL + 0), 0, wc);
-        if (ok) {
-          tc_fence_after();
-          issue_SP(dK_km, dQ_km, 0, tmem + C::TM_A);
-          mma_commit(bar(B_SFULL));
-          issue_SP(dV_km, dO_km, 0, tmem + C::TM_B);
-          mma_commit(bar(B_DPFULL));
-        }
-      }
-      for (int i = 0; i < nsteps && ok; ++i) {
-        const int st = i % C::QS;
-        const uint32_t par = i & 1;
-        ok = bounded_wait(bar(B_PFULL), par, wc);
+      bool ok = true;
+      int uc = 0, gs = 0;
+      for (int k = 0; ok; ++k) {
+        ok = bounded_wait(bar(B_UFULL + (k & 3)), (k >> 2) & 1, wc);
+        if (!ok) break;
+        const int u = s_queue[k & 3];
+        mbar_arrive(bar(B_UEMPTY + (k & 3)));
+        if (u < 0) break;
+        const Unit U = decode(u);
+        const int nsteps = U.nsteps;
+        if (nsteps == 0) continue;
+        // this unit's K - c in place, Q_0 loaded
+        ok = bounded_wait(bar(B_KC), uc & 1, wc);
+        if (ok) ok = bounded_wait(bar(B_QFULL + gs % C::QS), (gs / C::QS) & 1, wc);
         if (!ok) break;
         tc_fence_after();
-        issue_grad(dO_mn, st, C::TM_DV, 0, i == 0);
-        ok = bounded_wait(bar(B_DSFULL), par, wc);
+        issue_SP(dK_km, dQ_km, gs % C::QS, tmem + C::TM_A);
+        mma_commit(bar(B_SFULL));
+        // B: the previous unit's last dQ^T has been read out
+        if (gs > 0) {
+          ok = bounded_wait(bar(B_DQEMPTY), (gs - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        issue_SP(dV_km, dO_km, gs % C::QS, tmem + C::TM_B);
+        mma_commit(bar(B_DPFULL));
+        for (int i = 0; i < nsteps && ok; ++i) {
+          const int gi = gs + i;
+          const int st = gi % C::QS;
+          const uint32_t par = gi & 1;
+          const int st1 = (gi + 1) % C::QS;
+          const uint32_t ph1 = ((gi + 1) / C::QS) & 1;
+          ok = bounded_wait(bar(B_PFULL), par, wc);
+          // dV(0) and dK(0) start the accumulators afresh: the previous
+          // unit's epilogue must have read them out of TMEM
+          if (ok && i == 0 && uc > 0) ok = bounded_wait(bar(B_ACCEMPTY), (uc - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_grad(dO_mn, st, C::TM_DV, 0, i == 0);
+          if constexpr (C::EARLY_S) {
+            // dV(i)  S^T(i+1)  dQ^T(i)  dK(i)  dP^T(i+1)
+            if (i + 1 < nsteps) {
+              // S^T(i+1) over A: phase 1 has read S^T(i) and dV(i), issued
+              // before it, is the last reader of P^T(i)
+              ok = bounded_wait(bar(B_QFULL + st1), ph1, wc);
+              if (!ok) break;
+              tc_fence_after();
+              issue_SP(dK_km, dQ_km, st1, tmem + C::TM_A);
+              mma_commit(bar(B_SFULL));
+            }
+            // phase 2 has read dP^T(i) out of B and put dS^T(i) in shared memory
+            ok = bounded_wait(bar(B_DSFULL), par, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dq();
+            mma_commit(bar(B_DQFULL));
+            issue_dk_smem(st, i == 0);
+            mma_commit(bar(B_QEMPTY + st));
+          } else {
+            // dV(i)  dK(i)  S^T(i+1)  dQ^T(i)  dP^T(i+1)
+            ok = bounded_wait(bar(B_DSFULL), par, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_grad(dQ_mn, st, C::TM_DK, 16, i == 0);
+            mma_commit(bar(B_QEMPTY + st));
+            if (i + 1 < nsteps) {
+              ok = bounded_wait(bar(B_QFULL + st1), ph1, wc);
+              if (!ok) break;
+              tc_fence_after();
+              issue_SP(dK_km, dQ_km, st1, tmem + C::TM_A);
+              mma_commit(bar(B_SFULL));
+            }
+            issue_dq();
+            mma_commit(bar(B_DQFULL));
+          }
+          if (i + 1 < nsteps) {
+            ok = bounded_wait(bar(B_DQEMPTY), par, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_SP(dV_km, dO_km, st1, tmem + C::TM_B);
+            mma_commit(bar(B_DPFULL));
+          }
+        }
         if (!ok) break;
-        tc_fence_after();
-        issue_grad(dQ_mn, st, C::TM_DK, 16, i == 0);
-        mma_commit(bar(B_QEMPTY + st));
-        const int st1 = (i + 1) % C::QS;
-        if (i + 1 < nsteps) {
-          ok = bounded_wait(bar(B_QFULL + st1), ((i + 1) / C::QS) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-          issue_SP(dK_km, dQ_km, st1, tmem + C::TM_A);
-          mma_commit(bar(B_SFULL));
-        }
-        issue_dq();
-        mma_commit(bar(B_DQFULL));
-        if (i + 1 < nsteps) {
-          ok = bounded_wait(bar(B_DQEMPTY), par, wc);
-          if (!ok) break;
-          tc_fence_after();
-          issue_SP(dV_km, dO_km, st1, tmem + C::TM_B);
-          mma_commit(bar(B_DPFULL));
-        }
-      }
-      if (ok) {
+        // the unit's accumulators are final once its MMAs complete; this also
+        // releases K and V to the producer
         mma_commit(bar(B_FINAL));
-      } else {
+        gs += nsteps;
+        ++uc;
+      }
+      if (!ok) {
         mma_commit(bar(B_DRAIN));
         (void)drain_wait(bar(B_DRAIN), 0, p.err, kWaitLimitNs);
       }
@@ -922,171 +1091,213 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ------------------------------------------------ elementwise stage
     const int wg = warp >> 2;                      // query columns [64 wg, 64 wg + 64)
     const int r = threadIdx.x & 127;               // key row within the block = TMEM lane
-    const int kv = kv0 + r;
-    const bool kv_live = kv < p.Nk;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    bool ok = warp_wait_all(bar(B_KV), 0, wc);
-    if (ok) {
-      // K row r -> K - c in place (same swizzled layout; rows past Nk were
-      // zero-filled and stay zero).  Warpgroup wg takes chunks wg, wg + 2, ...
-      const float *cv = p.cvec + (size_t)bhkv * C::D;
-#pragma unroll 1
-      for (int ch = wg; ch < C::DCH; ch += 2) {
-        uint8_t *row = smem + C::OFF_K + ch * C::KV_CHUNK + r * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int col = ch * 64 + ((u ^ (r & 7)) << 3);
-          const float4 c_lo = *reinterpret_cast<const float4 *>(cv + col);
-          const float4 c_hi = *reinterpret_cast<const float4 *>(cv + col + 4);
-          const float cc[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
-          uint4 v = *reinterpret_cast<const uint4 *>(row + (u << 4));
-          uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
-            const float2 f = __bfloat1622float2(h2);
-            w[e] = kv_live ? pack_bf16x2(f.x - cc[2 * e], f.y - cc[2 * e + 1]) : 0u;
-          }
-          *reinterpret_cast<uint4 *>(row + (u << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_KC));
-    }
     const uint32_t tA = tmem + lane_off + C::TM_A;
     const uint32_t tB = tmem + lane_off + C::TM_B;
-    for (int i = 0; i < nsteps && ok; ++i) {
-      const int st = i % C::QS;
-      const uint32_t par = i & 1;
-      const int q0 = step_qblk(i) * C::BM;
-      ok = warp_wait_all(bar(B_QFULL + st), (i / C::QS) & 1, wc);
-      if (ok) ok = warp_wait_all(bar(B_SFULL), par, wc);
+    bool ok = true;
+    int uc = 0, gs = 0;
+    for (int k = 0; ok; ++k) {
+      ok = warp_wait_all(bar(B_UFULL + (k & 3)), (k >> 2) & 1, wc);
       if (!ok) break;
-      tc_fence_after();
-      // ---- phase 1: P^T for query columns [64 wg, 64 wg + 64), 16 at a time
-      uint32_t pkeep[4][8];
-      uint32_t keepbits[2] = {0u, 0u};               // dropout: bit c = column 64 wg + c kept
-      const uint32_t bhq = (uint32_t)(b * p.Hq + step_head(i));
-#pragma unroll
-      for (int sb = 0; sb < 4; ++sb) {
-        const int c0 = 64 * wg + 16 * sb;
-        uint32_t sv[16];
-        tmem_ld16(tA + c0, sv);
-        tmem_wait_ld();
-        const float4 *l4 = reinterpret_cast<const float4 *>(s_l2 + st * C::BM + c0);
-        // causal: key kv is hidden from query q when kv > q; key rows past
-        // Nk (zero-filled) are masked so they add nothing anywhere.  Query
-        // rows past Nq have L2 = +inf, so their P is 0.
-        const int first_vis = !kv_live ? 16 : (p.causal ? kv - (q0 + c0) : 0);
-        float pr[16];
-#pragma unroll
-        for (int e4 = 0; e4 < 4; ++e4) {
-          const float4 lq = l4[e4];
-          const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = 4 * e4 + u;
-            const float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[u]));
-            pr[c] = (c >= first_vis) ? pv : 0.f;
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pkeep[sb][e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
-        // P^T of query columns 32h + 16(sb%2) + [0,16) -> A columns 32h + 8(sb%2) + [0,8),
-        // all of which this thread has already read.  With dropout the dV
-        // operand is P^T * Z; pkeep keeps P^T for dS.
-        if (DROP) {
-          uint32_t m16 = 0;
-#pragma unroll
-          for (int gq = 0; gq < 4; ++gq)
-            m16 |= dropout_keep4(kv, q0 + c0 + 4 * gq, bhq, p, lane) << (4 * gq);
-          keepbits[sb >> 1] |= m16 << (16 * (sb & 1));
-          uint32_t pm[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            pm[e] = pack_bf16x2(((m16 >> (2 * e)) & 1u) ? pr[2 * e] : 0.f,
-                                ((m16 >> (2 * e + 1)) & 1u) ? pr[2 * e + 1] : 0.f);
-          tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 8 * (sb & 1), pm);
-        } else {
-          tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 8 * (sb & 1), pkeep[sb]);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_PFULL));
-      // ---- phase 2: dS^T = P^T (dP^T - D)
-      ok = warp_wait_all(bar(B_DPFULL), par, wc);
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll
-      for (int sb = 0; sb < 4; ++sb) {
-        const int c0 = 64 * wg + 16 * sb;
-        uint32_t dv[16];
-        tmem_ld16(tB + c0, dv);
-        tmem_wait_ld();
-        const float4 *d4 = reinterpret_cast<const float4 *>(s_dd + st * C::BM + c0);
-        uint32_t dk[8];
-#pragma unroll
-        for (int e4 = 0; e4 < 4; ++e4) {
-          const float4 dq4 = d4[e4];
-          const float dd[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
-          float ds[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = 4 * e4 + u;
-            const uint32_t pp = pkeep[sb][c >> 1];
-            const float pv = __uint_as_float((c & 1) ? (pp & 0xffff0000u) : (pp << 16));
-            float dpv = __uint_as_float(dv[c]);
-            if (DROP) dpv = ((keepbits[sb >> 1] >> (16 * (sb & 1) + c)) & 1u) ? dpv * p.drop_scale : 0.f;
-            ds[u] = pv * (dpv - dd[u]);
-          }
-          dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
-          dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
-        }
-        tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 16 + 8 * (sb & 1), dk);
-        // dS^T row r -> shared memory (B operand of the dQ^T MMA: 64-column
-        // chunks of 128-byte swizzled rows; 16-byte unit u of row r sits at
-        // unit u ^ (r % 8))
-        uint8_t *dsrow = smem + C::OFF_DS + (c0 >> 6) * C::DS_CHUNK + r * 128;
-        const int u0 = (c0 & 63) >> 3;
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          *reinterpret_cast<uint4 *>(dsrow + (((u0 + c) ^ (r & 7)) << 4)) =
-              make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_DSFULL));
-    }
-    // ------------------------------------------------------ epilogue
-    // warpgroup 0 writes dV, warpgroup 1 writes dK (one key row per thread)
-    if (ok) ok = warp_wait_all(bar(B_FINAL), 0, wc);
-    if (ok && nsteps > 0) {
-      tc_fence_after();
-      const size_t rowoff = ((size_t)bhkv * p.Nk + (kv_live ? kv : 0)) * C::D;
-      const uint32_t src = tmem + lane_off + (wg ? C::TM_DK : C::TM_DV);
-      __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + rowoff;
-      const float mul = wg ? p.scale : (DROP ? p.drop_scale : 1.f);
-#pragma unroll 1
-      for (int c = 0; c < C::D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(src + c * 32, v);
-        tmem_wait_ld();
-        uint32_t pkd[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pkd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+      const int u = s_queue[k & 3];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_UEMPTY + (k & 3)));
+      if (u < 0) break;
+      const Unit U = decode(u);
+      const int nsteps = U.nsteps;
+      const int kv = U.kv0 + r;
+      const bool kv_live = kv < p.Nk;
+      if (nsteps == 0) {
+        // no query row sees this key block: its gradients are zero
         if (kv_live) {
-          uint4 *o = reinterpret_cast<uint4 *>(dst + c * 32);
+          __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + ((size_t)U.bhkv * p.Nk + kv) * C::D;
+          for (int e = 0; e < C::D / 8; ++e) reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0, 0, 0, 0);
+        }
+        continue;
+      }
+      {
+        // K row r -> K - c in place (same swizzled layout; rows past Nk were
+        // zero-filled and stay zero).  Warpgroup wg takes the 16-byte units
+        // 4 wg .. 4 wg + 3 of each 128-byte chunk of the row; the entries of
+        // c they need are read before K has arrived.
+        const float *cv = p.cvec + (size_t)U.bhkv * C::D;
+        float cc[C::DCH][32];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+        for (int ch = 0; ch < C::DCH; ++ch)
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const int col = ch * 64 + (((4 * wg + e4) ^ (r & 7)) << 3);
+            const float4 c_lo = *reinterpret_cast<const float4 *>(cv + col);
+            const float4 c_hi = *reinterpret_cast<const float4 *>(cv + col + 4);
+            cc[ch][8 * e4 + 0] = c_lo.x; cc[ch][8 * e4 + 1] = c_lo.y;
+            cc[ch][8 * e4 + 2] = c_lo.z; cc[ch][8 * e4 + 3] = c_lo.w;
+            cc[ch][8 * e4 + 4] = c_hi.x; cc[ch][8 * e4 + 5] = c_hi.y;
+            cc[ch][8 * e4 + 6] = c_hi.z; cc[ch][8 * e4 + 7] = c_hi.w;
+          }
+        ok = warp_wait_all(bar(B_KV), uc & 1, wc);
+        if (!ok) break;
+#pragma unroll
+        for (int ch = 0; ch < C::DCH; ++ch) {
+          uint8_t *row = smem + C::OFF_K + ch * C::KV_CHUNK + r * 128;
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const int e8 = 4 * wg + e4;
+            uint4 v = *reinterpret_cast<const uint4 *>(row + (e8 << 4));
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+              const float2 f = __bfloat1622float2(h2);
+              w[e] = kv_live ? pack_bf16x2(f.x - cc[ch][8 * e4 + 2 * e], f.y - cc[ch][8 * e4 + 2 * e + 1])
+                             : 0u;
+            }
+            *reinterpret_cast<uint4 *>(row + (e8 << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(B_KC));
+      }
+      for (int i = 0; i < nsteps && ok; ++i) {
+        const int gi = gs + i;
+        const int st = gi % C::QS;
+        const uint32_t par = gi & 1;
+        const int q0 = step_qblk(U, i) * C::BM;
+        ok = warp_wait_all(bar(B_QFULL + st), (gi / C::QS) & 1, wc);
+        if (ok) ok = warp_wait_all(bar(B_SFULL), par, wc);
+        if (!ok) break;
+        tc_fence_after();
+        // ---- phase 1: P^T for query columns [64 wg, 64 wg + 64), 16 at a time
+        uint32_t pkeep[4][8];
+        uint32_t keepbits[2] = {0u, 0u};               // dropout: bit c = column 64 wg + c kept
+        const uint32_t bhq = (uint32_t)(U.b * p.Hq + step_head(U, i));
+#pragma unroll
+        for (int sb = 0; sb < 4; ++sb) {
+          const int c0 = 64 * wg + 16 * sb;
+          uint32_t sv[16];
+          tmem_ld16(tA + c0, sv);
+          tmem_wait_ld();
+          const float4 *l4 = reinterpret_cast<const float4 *>(s_l2 + st * C::BM + c0);
+          // causal: key kv is hidden from query q when kv > q; key rows past
+          // Nk (zero-filled) are masked so they add nothing anywhere.  Query
+          // rows past Nq have L2 = +inf, so their P is 0.
+          const int first_vis = !kv_live ? 16 : (p.causal ? kv - (q0 + c0) : 0);
+          float pr[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 lq = l4[e4];
+            const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 4 * e4 + e;
+              const float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[e]));
+              pr[c] = (c >= first_vis) ? pv : 0.f;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pkeep[sb][e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+          // P^T of query columns 32h + 16(sb%2) + [0,16) -> A columns 32h + 8(sb%2) + [0,8),
+          // all of which this thread has already read.  With dropout the dV
+          // operand is P^T * Z; pkeep keeps P^T for dS.
+          if (DROP) {
+            uint32_t m16 = 0;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq)
+              m16 |= dropout_keep4(kv, q0 + c0 + 4 * gq, bhq, p, lane) << (4 * gq);
+            keepbits[sb >> 1] |= m16 << (16 * (sb & 1));
+            uint32_t pm[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              pm[e] = pack_bf16x2(((m16 >> (2 * e)) & 1u) ? pr[2 * e] : 0.f,
+                                  ((m16 >> (2 * e + 1)) & 1u) ? pr[2 * e + 1] : 0.f);
+            tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 8 * (sb & 1), pm);
+          } else {
+            tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 8 * (sb & 1), pkeep[sb]);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL));
+        // ---- phase 2: dS^T = P^T (dP^T - D)
+        ok = warp_wait_all(bar(B_DPFULL), par, wc);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int sb = 0; sb < 4; ++sb) {
+          const int c0 = 64 * wg + 16 * sb;
+          uint32_t dv[16];
+          tmem_ld16(tB + c0, dv);
+          tmem_wait_ld();
+          const float4 *d4 = reinterpret_cast<const float4 *>(s_dd + st * C::BM + c0);
+          uint32_t dk[8];
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 dq4 = d4[e4];
+            const float dd[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
+            float ds[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 4 * e4 + e;
+              const uint32_t pp = pkeep[sb][c >> 1];
+              const float pv = __uint_as_float((c & 1) ? (pp & 0xffff0000u) : (pp << 16));
+              float dpv = __uint_as_float(dv[c]);
+              if (DROP) dpv = ((keepbits[sb >> 1] >> (16 * (sb & 1) + c)) & 1u) ? dpv * p.drop_scale : 0.f;
+              ds[e] = pv * (dpv - dd[e]);
+            }
+            dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+            dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
+          }
+          // dS^T -> A (the dK operand) unless EARLY_S, where S^T(i+1) may
+          // already be there and dK reads dS^T from shared memory
+          if constexpr (!C::EARLY_S) tmem_st8(tA + 32 * (2 * wg + (sb >> 1)) + 16 + 8 * (sb & 1), dk);
+          // dS^T row r -> shared memory (B operand of the dQ^T MMA, and with
+          // EARLY_S the A operand of dK: 64-column chunks of 128-byte swizzled
+          // rows; 16-byte unit u of row r sits at unit u ^ (r % 8))
+          uint8_t *dsrow = smem + C::OFF_DS + (c0 >> 6) * C::DS_CHUNK + r * 128;
+          const int u0 = (c0 & 63) >> 3;
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            *reinterpret_cast<uint4 *>(dsrow + (((u0 + c) ^ (r & 7)) << 4)) =
+                make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_DSFULL));
+      }
+      if (!ok) break;
+      // ---------------------------------------------------- epilogue
+      // warpgroup 0 writes dV, warpgroup 1 writes dK (one key row per thread);
+      // the accumulators are released once read, before the stores complete
+      ok = warp_wait_all(bar(B_FINAL), uc & 1, wc);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const size_t rowoff = ((size_t)U.bhkv * p.Nk + (kv_live ? kv : 0)) * C::D;
+        const uint32_t src = tmem + lane_off + (wg ? C::TM_DK : C::TM_DV);
+        __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + rowoff;
+        const float mul = wg ? p.scale : (DROP ? p.drop_scale : 1.f);
+#pragma unroll 1
+        for (int c = 0; c < C::D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(src + c * 32, v);
+          tmem_wait_ld();
+          if (c == C::D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(B_ACCEMPTY));
+          }
+          uint32_t pkd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pkd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+          if (kv_live) {
+            uint4 *o = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+          }
         }
       }
-    } else if (ok && nsteps == 0 && kv_live) {
-      // no query row sees this key block: its gradients are zero
-      __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + ((size_t)bhkv * p.Nk + kv) * C::D;
-      for (int e = 0; e < C::D / 8; ++e) reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0, 0, 0, 0);
+      gs += nsteps;
+      ++uc;
     }
   } else if (warp < C::PRODUCER_WARP) {
     // ------------------------------------------------ dQ^T readout
@@ -1094,28 +1305,41 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int t = quad * 32 + lane;                  // TMEM lane = row d of dQ^T
     const int ch0 = ((warp - C::READOUT_WARP0) >> 2) * 2;   // chunks ch0, ch0 + 1
     const uint32_t src = tmem + ((uint32_t)(quad * 32) << 16) + C::TM_B + ch0 * 32;
-    for (int i = 0; i < nsteps; ++i) {
-      if (!warp_wait_all(bar(B_DQFULL), i & 1, wc)) break;
-      tc_fence_after();
-      uint32_t v0[32], v1[32];
-      const bool live_rows = quad * 32 < C::D;    // d = 64: lanes 64..127 carry no dQ
-      if (live_rows) {
-        tmem_ld32(src, v0);
-        tmem_ld32(src + 32, v1);
-        tmem_wait_ld();
+    const bool live_rows = quad * 32 < C::D;    // d = 64: lanes 64..127 carry no dQ
+    bool ok = true;
+    int gs = 0;
+    for (int k = 0; ok; ++k) {
+      ok = warp_wait_all(bar(B_UFULL + (k & 3)), (k >> 2) & 1, wc);
+      if (!ok) break;
+      const int u = s_queue[k & 3];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_UEMPTY + (k & 3)));
+      if (u < 0) break;
+      const Unit U = decode(u);
+      for (int i = 0; i < U.nsteps; ++i) {
+        ok = warp_wait_all(bar(B_DQFULL), (gs + i) & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
+        if (live_rows) {
+          tmem_ld32(src, v0);
+          tmem_ld32(src + 32, v1);
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_DQEMPTY));
+        if (!live_rows) continue;
+        const int h = step_head(U, i), q0 = step_qblk(U, i) * C::BM;
+        const int nvalid = min(C::BM, p.Nq - q0);
+        float *acc = p.dq_acc + (((size_t)(U.b * p.Hq + h)) * p.Nq + q0 + ch0 * 32) * C::D + t;
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (ch0 * 32 + c < nvalid) atomicAdd(acc + (size_t)c * C::D, __uint_as_float(v0[c]));
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (ch0 * 32 + 32 + c < nvalid) atomicAdd(acc + (size_t)(32 + c) * C::D, __uint_as_float(v1[c]));
       }
-      tc_fence_before();
-      mbar_arrive(bar(B_DQEMPTY));
-      if (!live_rows) continue;
-      const int h = step_head(i), q0 = step_qblk(i) * C::BM;
-      const int nvalid = min(C::BM, p.Nq - q0);
-      float *acc = p.dq_acc + (((size_t)(b * p.Hq + h)) * p.Nq + q0 + ch0 * 32) * C::D + t;
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (ch0 * 32 + c < nvalid) atomicAdd(acc + (size_t)c * C::D, __uint_as_float(v0[c]));
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (ch0 * 32 + 32 + c < nvalid) atomicAdd(acc + (size_t)(32 + c) * C::D, __uint_as_float(v1[c]));
+      gs += U.nsteps;
     }
   }
 
@@ -1131,8 +1355,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // integers (f32).  One CTA per (batch, key/value head), one thread per column.
 template <int D>
 __global__ void bwd_center_kernel(const __nv_bfloat16 *__restrict__ k, float *__restrict__ cvec,
-                                  int Nk) {
+                                  int Nk, int *__restrict__ sched) {
   const int t = threadIdx.x;
+  if (blockIdx.x == 0 && t == 0) *sched = 0;   // work counter of the dK/dV kernel
   const __nv_bfloat16 *kh = k + (size_t)blockIdx.x * Nk * D + t;
   const int nr = min(Nk, kCenterRows);
   float acc = 0.f;
@@ -1232,19 +1457,21 @@ bool make_map(CUtensorMap *m, const void *base, int rows_per_head, int heads, in
 
 struct WsPtrs {
   float *dsum, *l2, *cvec, *dq_acc;
+  int *sched;
 };
 WsPtrs ws_ptrs(const AttnArgs &a) {
   char *w = (char *)a.ws;
   return {(float *)w, (float *)(w + ws_l2_offset(a.B, a.Hq, a.Nq)),
           (float *)(w + ws_c_offset(a.B, a.Hq, a.Nq)),
-          (float *)(w + ws_dq_offset(a.B, a.Hq, a.Nq, a.d))};
+          (float *)(w + ws_dq_offset(a.B, a.Hq, a.Nq, a.d)),
+          (int *)(w + ws_sched_offset(a.B, a.Hq, a.Nq, a.d))};
 }
 
 template <int D>
 int run_prep(const AttnArgs &a) {
   const WsPtrs w = ws_ptrs(a);
   bwd_center_kernel<D><<<(unsigned)(a.B * a.Hkv), D, 0, a.stream>>>(
-      (const __nv_bfloat16 *)a.k, w.cvec, a.Nk);
+      (const __nv_bfloat16 *)a.k, w.cvec, a.Nk, w.sched);
   if (cudaGetLastError() != cudaSuccess) return 5;
   const int npad = (int)ws_npad(a.Nq);
   const long long prows = (long long)a.B * a.Hq * npad;
@@ -1271,6 +1498,7 @@ int run_dkdv(const AttnArgs &a) {
   p.dsum = w.dsum;
   p.cvec = w.cvec;
   p.dq_acc = w.dq_acc;
+  p.sched = w.sched;
   p.dk = (__nv_bfloat16 *)a.dk;
   p.dv = (__nv_bfloat16 *)a.dv;
   p.Hq = a.Hq; p.Hkv = a.Hkv; p.Nq = a.Nq; p.Nk = a.Nk;
@@ -1278,6 +1506,15 @@ int run_dkdv(const AttnArgs &a) {
   p.nqb = (a.Nq + C::BM - 1) / C::BM;
   p.nkb = (a.Nk + C::BN - 1) / C::BN;
   p.BHkv = a.B * a.Hkv;
+  {
+    // causal unit order: groups of key/value heads whose f32 dQ accumulator
+    // and Q, dO tiles (g query heads each) take about BWD_GROUP_BYTES, so the
+    // reductions of a group stay in L2; inside a group the heaviest key
+    // blocks first.  Non-causal units are all equal: head by head.
+    const double per_kv_head = (double)(a.Hq / a.Hkv) * a.Nq * a.d * 8.0;
+    const double hg = floor((double)BWD_GROUP_BYTES / per_kv_head);
+    p.hg = !a.causal || hg < 1.0 ? 1 : (hg >= (double)p.BHkv ? p.BHkv : (int)hg);
+  }
   p.scale = a.scale;
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
@@ -1294,7 +1531,13 @@ int run_dkdv(const AttnArgs &a) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
       return 5;
-    kern<<<(unsigned)units, C::THREADS, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
+    // persistent: one CTA per SM (at most one per unit)
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 5;
+    const long long grid = (BWD_PERSIST && units > sms) ? sms : units;
+    kern<<<(unsigned)grid, C::THREADS, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
   } else {
     if (a.drop_thr != 0) return 2;   // dropout runs in the wide kernel only (d <= 128)
     auto kern = bwd_kernel<C>;
@@ -1332,8 +1575,8 @@ int launch_bwd_prep_bf16(const AttnArgs &a) {
 // 8-11% slower than bwd_wide_kernel at d = 64 and 128.)
 int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {
-    case 64: return run_dkdv<BwdWideCfg<64, 4>, true>(a);
-    case 128: return run_dkdv<BwdWideCfg<128, 2>, true>(a);
+    case 64: return run_dkdv<BwdWideCfg<64, 4, true>, true>(a);
+    case 128: return run_dkdv<BwdWideCfg<128, 2, false>, true>(a);
     case 256: {
       int st = run_dkdv<BwdCfg<256, kDV, 64, 2, 2>, false>(a);
       return st ? st : run_dkdv<BwdCfg<256, kDKDQ, 64, 1, 1>, false>(a);

@@ -37,14 +37,18 @@ struct AttnArgs {
 //   L2  [B*Hq][Npad]   log2e * L - scale*log2e * (q . c): the log-sum-exp in
 //                      base 2, shifted for the centred K; rows past Nq +inf
 //   c   [B*Hq][d]      per key/value head centring vector (first B*Hkv*d used)
+//   n   int32          work counter of the persistent dK/dV kernel (zeroed by prep)
 //   dQ  [B*Hq][Nq][d]  dQ accumulator, 256-byte aligned
 // Npad = Nq rounded up to 128, so every 64- or 128-row query block of D and
 // L2 is a 256-byte aligned block a bulk copy can fetch.
 inline size_t ws_npad(int Nq) { return (size_t)((Nq + 127) / 128) * 128; }
 inline size_t ws_l2_offset(int B, int Hq, int Nq) { return (size_t)B * Hq * ws_npad(Nq) * 4; }
 inline size_t ws_c_offset(int B, int Hq, int Nq) { return 2 * ws_l2_offset(B, Hq, Nq); }
+inline size_t ws_sched_offset(int B, int Hq, int Nq, int d) {
+  return ws_c_offset(B, Hq, Nq) + (size_t)B * Hq * d * 4;
+}
 inline size_t ws_dq_offset(int B, int Hq, int Nq, int d) {
-  return (ws_c_offset(B, Hq, Nq) + (size_t)B * Hq * d * 4 + 255) & ~(size_t)255;
+  return (ws_sched_offset(B, Hq, Nq, d) + 16 + 255) & ~(size_t)255;
 }
 inline size_t ws_bytes(int B, int Hq, int Nq, int d) {
   return ws_dq_offset(B, Hq, Nq, d) + (size_t)B * Hq * Nq * d * 4;

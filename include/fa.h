@@ -167,9 +167,10 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd and fa_bwd_f32
  * need (float32 throughout): the per-row vector D = rowsum(dO * O) and the
  * per-row base-2 log-sum-exp used by the backward, each padded to a multiple
- * of 64 rows per head; one centring vector per head (B*Hq*d); and a dQ
- * accumulator (B*Hq*Nq*d), 256-byte aligned.  About 4*B*Hq*(Nq*(d+2) + d)
- * bytes.  Returns 0 for invalid sizes.
+ * of 128 rows per head; one centring vector per head (B*Hq*d); a work
+ * counter of the persistent main pass; and a dQ accumulator (B*Hq*Nq*d),
+ * 256-byte aligned.  About 4*B*Hq*(Nq*(d+2) + d) + 256 bytes.  Returns 0 for
+ * invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
 
@@ -192,9 +193,12 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
  *   fa_bwd_prep  -- per key/value head the centring vector c (the mean of its
  *                   first 64 key rows, rounded to integers); per query row
  *                   D = rowsum(dout * o) and the base-2 log-sum-exp shifted
- *                   by scale * q . c; the dQ accumulator zeroed;
+ *                   by scale * q . c; the dQ accumulator and the main pass's
+ *                   work counter zeroed;
  *   fa_bwd_dkdv  -- the main pass: dk, dv written, dQ accumulated (f32) in
- *                   the workspace;
+ *                   the workspace.  Needs fa_bwd_prep on the same workspace
+ *                   before every call (d = 64 and 128 hand out work units
+ *                   through the counter prep zeroes);
  *   fa_bwd_dq    -- dq = bf16(scale * accumulator).
  * Same argument rules as fa_bwd.
  */

@@ -46,8 +46,10 @@ def test_strerror_covers_codes():
 
 
 def _ws_expected(B, H, N, d):
+    # D and L2 rows padded to 128 per head, the centring vectors, a 16-byte
+    # work counter, then the 256-byte aligned f32 dQ accumulator
     npad = (N + 127) // 128 * 128
-    head = 2 * B * H * npad * 4 + B * H * d * 4
+    head = 2 * B * H * npad * 4 + B * H * d * 4 + 16
     return (head + 255) // 256 * 256 + B * H * N * d * 4
 
 
