@@ -208,7 +208,7 @@ __device__ __forceinline__ void reduce_dq_chunk(const uint32_t (&v)[32], float *
     if (cq + c < nvalid) atomicAdd(a + (size_t)c * C::D, __uint_as_float(v[c]));
 }
 
-template <class C>
+template <class C, bool DROP>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -538,6 +538,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // rows past Nq have L2 = +inf, so their P is 0.
         const int first_vis = !kv_live ? 32 : (p.causal ? kv - q0 : 0);
         const bool unmasked = __all_sync(0xffffffffu, first_vis <= 0);
+        // dropout: bit c = query column q0 + c kept for this key row (the same
+        // Philox words the forward used); the dV pass stores P^T * Z, the dK /
+        // dQ pass scales the kept dP^T by 1 / (1 - p)
+        uint32_t keep = 0xffffffffu;
+        if (DROP) {
+          keep = 0u;
+          const uint32_t bhq = (uint32_t)(b * p.Hq + step_head(i));
+#pragma unroll
+          for (int gq = 0; gq < 8; ++gq) keep |= dropout_keep4(kv, q0 + 4 * gq, bhq, p, lane) << (4 * gq);
+        }
         uint32_t pk[16], dk[16];
         auto body = [&](auto masked_tag) {
           constexpr bool MASKED = decltype(masked_tag)::value;
@@ -553,8 +563,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int c = 4 * e4 + u;
               float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[u]));
               if (MASKED) pv = (c >= first_vis) ? pv : 0.f;
-              pr[u] = pv;
-              ds[u] = C::HAS_DP ? pv * (__uint_as_float(dv[c]) - dvv[u]) : 0.f;
+              const bool kept = !DROP || ((keep >> c) & 1u);
+              pr[u] = kept ? pv : 0.f;
+              float dpv = __uint_as_float(dv[c]);
+              if (DROP) dpv = kept ? dpv * p.drop_scale : 0.f;
+              ds[u] = C::HAS_DP ? pv * (dpv - dvv[u]) : 0.f;
             }
             pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
             pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
@@ -611,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t rowoff = ((size_t)bhkv * p.Nk + (kv_live ? kv : 0)) * C::D;
       const uint32_t src = tmem + lane_off + (wg ? C::TM_DK : C::TM_DV);
       __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + rowoff;
-      const float mul = wg ? p.scale : 1.f;
+      const float mul = wg ? p.scale : (DROP ? p.drop_scale : 1.f);
 #pragma unroll 1
       for (int c = 0; c < C::D / 32; ++c) {
         uint32_t v[32];
@@ -1539,8 +1552,7 @@ int run_dkdv(const AttnArgs &a) {
     const long long grid = (BWD_PERSIST && units > sms) ? sms : units;
     kern<<<(unsigned)grid, C::THREADS, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
   } else {
-    if (a.drop_thr != 0) return 2;   // dropout runs in the wide kernel only (d <= 128)
-    auto kern = bwd_kernel<C>;
+    auto kern = a.drop_thr != 0 ? bwd_kernel<C, true> : bwd_kernel<C, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
       return 5;

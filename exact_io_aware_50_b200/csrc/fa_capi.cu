@@ -302,7 +302,7 @@ FA_EXPORT int fa_bwd_dropout(const void *q, const void *k, const void *v, const 
   int st = fa::dropout_params(p_drop, seed, offset, a);
   if (st) return st;
   if ((st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal))) return st;
-  if (d != 64 && d != 128 && !(d == 256 && a.drop_thr == 0)) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   const void *ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
   for (const void *p : ptrs)
     if (!fa::aligned16(p)) return FA_ERR_ALIGNMENT;

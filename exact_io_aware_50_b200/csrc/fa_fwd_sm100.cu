@@ -64,7 +64,8 @@
 //   it (p_empty, which also orders the rare O~ rescale after that MMA), and
 //   P_t(j) V_j runs SMEM x SMEM.  Issue order per block: S0(j+1), S1(j+1),
 //   PV0(j), PV1(j); the producer loads K one block ahead of V.
-// * P in TMEM (d = 256 bf16): P overwrites the upper half of S_t's columns;
+// * P in TMEM (kept as an option, no instance uses it now): P overwrites the
+//   upper half of S_t's columns;
 //   issue order PV0(j), S0(j+1), PV1(j), S1(j+1), so the softmax of one tile
 //   overlaps the tensor-core work of the other.  tcgen05 ops of one thread
 //   complete in issue order, and tcgen05.commit arrives after all earlier
@@ -887,7 +888,7 @@ int launch_fwd_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {
     case 64: return run_fwd<FwdCfg<64, 2, 128, 3, 2, true>>(a);
     case 128: return run_fwd<FwdCfg<128, 2, 128, 1, 2, true>>(a);
-    case 256: return run_fwd<FwdCfg<256, 1, 128, 1>>(a);
+    case 256: return run_fwd<FwdCfg<256, 1, 128, 1, 2, true>>(a);
     default: return 2;
   }
 }

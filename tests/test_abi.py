@@ -153,7 +153,7 @@ def test_dropout_argument_errors():
         assert bwd(bad) == F.FA_ERR_INVALID_ARG
     assert fwd(0.1, ptrs=(0,) + (FAKE,) * 4) == F.FA_ERR_INVALID_ARG
     assert fwd(0.1, d=96) == F.FA_ERR_UNSUPPORTED
-    assert bwd(0.1, d=256) == F.FA_ERR_UNSUPPORTED      # dropout backward: d = 64, 128
+    assert bwd(0.1, d=96) == F.FA_ERR_UNSUPPORTED       # dropout backward: d = 64, 128, 256
     assert fwd(0.1, ptrs=(FAKE + 2,) + (FAKE,) * 4) == F.FA_ERR_ALIGNMENT
 
 

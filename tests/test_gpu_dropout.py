@@ -47,7 +47,8 @@ def test_dropout_mask_bits():
 
 
 CASES = [(1, 2, 1, 300, 64, True, 0.1), (2, 2, 2, 257, 128, False, 0.5),
-         (1, 4, 2, 513, 128, True, 0.3)]
+         (1, 4, 2, 513, 128, True, 0.3), (1, 2, 1, 300, 256, True, 0.2),
+         (2, 2, 2, 200, 256, False, 0.4)]
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "x".join(str(v) for v in c))
