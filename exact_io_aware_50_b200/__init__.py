@@ -11,5 +11,5 @@ from .binding import (  # noqa: F401
     fa_fwd_fp8, forward_fp8,
     fa_fwd_dropout, fa_bwd_dropout, forward_dropout, backward_dropout,
     fa_bwd_workspace_size, fa_bwd_prep, fa_bwd_dkdv, fa_bwd_dq, fa_device_status,
-    fa_wait_selftest, fa_exp2_eval, fa_strerror, forward, forward_splitkv, backward,
+    fa_wait_selftest, fa_strerror, forward, forward_splitkv, backward,
 )

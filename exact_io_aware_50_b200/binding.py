@@ -29,7 +29,7 @@ EXPORTS = ("fa_fwd", "fa_fwd_fp8", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_s
            "fa_fwd_splitkv_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prep",
            "fa_bwd_dkdv",
            "fa_bwd_dq", "fa_fwd_f32", "fa_bwd_f32", "fa_device_status", "fa_wait_selftest",
-           "fa_exp2_eval", "fa_strerror")
+           "fa_strerror")
 
 
 class FaError(RuntimeError):
@@ -81,8 +81,6 @@ def lib():
         L.fa_device_status.restype = I
         L.fa_wait_selftest.argtypes = [ctypes.c_longlong, P]
         L.fa_wait_selftest.restype = I
-        L.fa_exp2_eval.argtypes = [P, P, I, I, P]
-        L.fa_exp2_eval.restype = I
         L.fa_strerror.argtypes = [I]
         L.fa_strerror.restype = ctypes.c_char_p
         _lib = L
@@ -164,10 +162,6 @@ def fa_device_status(stream=0):
 
 def fa_wait_selftest(timeout_ns, stream=0):
     return lib().fa_wait_selftest(int(timeout_ns), stream)
-
-
-def fa_exp2_eval(x, y, n, poly, stream=0):
-    return lib().fa_exp2_eval(x, y, n, int(poly), stream)
 
 
 def fa_strerror(status):

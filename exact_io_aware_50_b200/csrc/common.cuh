@@ -225,7 +225,7 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
-// The same two forms for 8-bit operands (kind::f8f6f4: K = 32 per
+// The shared-memory form for 8-bit operands (kind::f8f6f4: K = 32 per
 // instruction, 32 bytes of a K-major row as in the 16-bit kinds).
 __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -234,16 +234,6 @@ __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -407,27 +397,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x evaluated on the FMA pipe (the MUFU unit that runs ex2 is the
-// softmax's bottleneck, so part of the exponentials go here instead).
-// Range reduction: x = j + f with j the nearest integer -- adding 1.5 * 2^23
-// leaves j in the low mantissa bits of t -- and f in [-1/2, 1/2].  2^f comes
-// from a cubic 1 + f (c1 + f (c2 + f c3)) fitted for minimum relative error
-// on [-1/2, 1/2] with the constant term held at 1, so 2^x is exact at every
-// integer x -- in particular at the row maximum, where x = 0 (maximum
-// relative error 1.02e-4, below bf16 resolution) -- and 2^j is applied by
-// adding j to the exponent field.  Valid for x <= 127; inputs below -126
-// (including -inf) return a value below 2^-125 instead of 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float j = t - 12582912.0f;
-  const float f = x - j;
-  float p = fmaf(0.055008817464113235f, f, 0.24221080541610718f);
-  p = fmaf(p, f, 0.6932829022407532f);
-  p = fmaf(p, f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {

@@ -60,13 +60,12 @@
 namespace fa {
 namespace {
 
-// bwd_kernel warp roles: 0-7 elementwise stage (two warpgroups, half of the
-// query columns each, 32 at a time; each also reads out and reduces a quarter
-// of dQ^T when a step has four 32-column chunks), 8-11 dQ readout, 12 TMA
-// producer, 13 MMA issuer.  The producer and MMA roles run in lane 0 alone
-// (measured ~8% faster on B200 than keeping the warp converged around each
-// wait).  Its single-pass mode (kFull) serves d <= 128 when selected; the
-// library launches bwd_wide_kernel there instead.
+// bwd_kernel (d = 256, two passes) warp roles: 0-7 elementwise stage (two
+// warpgroups, half of the query columns each, 32 at a time; each also reads
+// out and reduces a quarter of dQ^T when a step has four 32-column chunks),
+// 8-11 dQ readout, 12 TMA producer, 13 MMA issuer.  The producer and MMA roles
+// run in lane 0 alone (measured ~8% faster on B200 than keeping the warp
+// converged around each wait).
 constexpr int kThreads = 448;
 constexpr int kReadoutWarp0 = 8;
 constexpr int kProducerWarp = 12;
@@ -74,7 +73,7 @@ constexpr int kMmaWarp = 13;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kCenterRows = 64;   // key rows averaged into the centring vector c
 
-enum Mode { kFull = 0, kDV = 1, kDKDQ = 2 };
+enum Mode { kDV = 1, kDKDQ = 2 };   // the dV pass, then the dK and dQ pass
 
 // BM_ query rows per step (MMA N), NSETS_ TMEM score sets, QS_ depth of the
 // Q/dO ring.  An M = 128 tcgen05 MMA takes about as long for N = 64 as for
@@ -88,8 +87,6 @@ struct BwdCfg {
   static constexpr int NSETS = NSETS_;
   static constexpr int QS = QS_;
   static_assert(BM == 64 || BM == 128, "query block");
-  // dQ^T is written over the dP^T columns (full pass) or into its own columns
-  static constexpr bool DQ_IN_DP = MODE == kFull;
   static constexpr bool HAS_DP = MODE != kDV;
   static constexpr bool HAS_DV = MODE != kDKDQ;
   static constexpr bool HAS_DK = MODE != kDV;
@@ -118,18 +115,17 @@ struct BwdCfg {
   // so no alignment slack is reserved.
   static constexpr int SMEM = OFF_MISC + 16;
   // TMEM columns (a "set" holds the scores of one step).
-  //   kFull : dV [0, D), dK [D, 2D), set at 2D: S^T [0,128) dP^T [128,256);
-  //           after the elementwise stage, for query columns 32h..32h+31:
-  //           P^T at [32h, 32h+16), dS^T at [32h+16, 32h+32); dQ^T [128,256)
-  //   kDV   : dV [0, 256), set x at 256 + 64x: S^T [0,64); then P^T as above
+  //   kDV   : dV [0, 256), set x at 256 + 64x: S^T [0,64); after the
+  //           elementwise stage, for query columns 32h..32h+31, P^T at
+  //           [32h, 32h+16)
   //   kDKDQ : dK [0, 256), set at 256: S^T [0,64) dP^T [64,128); then dS^T
-  //           as above, dQ^T halves [128,192) and [192,256)
+  //           at [32h+16, 32h+32), dQ^T halves [128,192) and [192,256)
   static constexpr int TM_DV = 0;
-  static constexpr int TM_DK = MODE == kFull ? D : 0;
-  static constexpr int TM_SET0 = MODE == kFull ? 2 * D : D;
+  static constexpr int TM_DK = 0;
+  static constexpr int TM_SET0 = D;
   static constexpr int SET_STRIDE = MODE == kDV ? BM : 2 * BM;
   static constexpr int TM_DP = BM;                          // dP^T offset inside a set
-  static constexpr int TM_DQ = MODE == kFull ? BM : 128;    // dQ^T offset inside a set
+  static constexpr int TM_DQ = 128;                         // dQ^T offset inside a set
   static constexpr int NHALF = D == 256 ? 2 : 1;            // dQ^T pieces of 128 rows of d
   static constexpr int NCH = NHALF * BM / 32;               // 32-column chunks of dQ^T
   // the readout warpgroup reads dQ^T chunks 0, 1; the elementwise warpgroups
@@ -138,8 +134,7 @@ struct BwdCfg {
   static constexpr int TM_ALLOC = 512;
   static_assert(TM_SET0 + NSETS * SET_STRIDE + (MODE == kDKDQ ? 128 : 0) <= TM_ALLOC, "TMEM");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(MODE != kFull || D <= 128, "full pass needs d <= 128");
-  static_assert(MODE == kFull || D == 256, "split passes are for d = 256");
+  static_assert(D == 256, "the two passes are for d = 256");
   // with two score sets, S^T(i+1) is issued before step i's gradients release
   // Q_i / dO_i, so the ring needs a second slot
   static_assert(NSETS == 1 || QS >= 2, "two score sets need two Q/dO slots");
@@ -435,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ok = bounded_wait(bar(B_PFULL + x), set_phase(i), wc);
       if (!ok) break;
-      if (C::HAS_DQ && C::NSETS == 1 && !C::DQ_IN_DP && i >= 1) {
+      if (C::HAS_DQ && C::NSETS == 1 && i >= 1) {
         ok = bounded_wait(bar(B_DQEMPTY + x), set_phase(i - 1), wc);
         if (!ok) break;
       }
@@ -450,18 +445,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (C::NSETS == 1 && i + 1 < nsteps) {
         // S^T(i+1) only overwrites P^T/dS^T, which dV/dK(i) (issued earlier)
-        // consume in order; dP^T(i+1) overwrites dQ^T(i) when they share
-        // columns, so it waits for the readout of dQ^T(i).
+        // consume in order
         const int st1 = (i + 1) % C::QS;
         ok = bounded_wait(bar(B_QFULL + st1), ((i + 1) / C::QS) & 1, wc);
         if (!ok) break;
         tc_fence_after();
         issue_S(x, st1);
-        if (C::HAS_DQ && C::DQ_IN_DP) {
-          ok = bounded_wait(bar(B_DQEMPTY + x), set_phase(i), wc);
-          if (!ok) break;
-          tc_fence_after();
-        }
         {
           issue_dP(x, st1);
           mma_commit(bar(B_SFULL + x));

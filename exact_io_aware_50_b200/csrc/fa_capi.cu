@@ -104,18 +104,6 @@ int validate_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, i
 
 int device_prologue(int *dev, AttnArgs &a) { return prologue(dev, a); }
 
-namespace {
-__global__ void exp2_eval_kernel(const float *x, float *y, int n, int poly) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = poly ? exp2_poly(x[i]) : fast_exp2(x[i]);
-}
-}  // namespace
-
-int launch_exp2_eval(const float *x, float *y, int n, int poly, cudaStream_t stream) {
-  exp2_eval_kernel<<<(n + 255) / 256, 256, 0, stream>>>(x, y, n, poly);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
 int launch_wait_selftest(long long timeout_ns, cudaStream_t stream, unsigned *err) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>(timeout_ns, err);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -428,16 +416,6 @@ FA_EXPORT int fa_device_status(fa_stream_t stream) {
     return FA_ERR_CUDA;
   if (host & fa::kErrTimeout) return FA_ERR_TIMEOUT;
   return host ? FA_ERR_CUDA : FA_OK;
-}
-
-FA_EXPORT int fa_exp2_eval(const float *x, float *y, int n, int poly, fa_stream_t stream) {
-  if (!x || !y || n < 0) return FA_ERR_INVALID_ARG;
-  if (n == 0) return FA_OK;
-  AttnArgs a;
-  int dev;
-  int st = fa::prologue(&dev, a);
-  if (st) return st;
-  return fa::launch_exp2_eval(x, y, n, poly, (cudaStream_t)stream);
 }
 
 FA_EXPORT int fa_wait_selftest(long long timeout_ns, fa_stream_t stream) {

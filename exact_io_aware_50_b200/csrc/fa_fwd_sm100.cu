@@ -56,21 +56,16 @@
 // taken out of L.  The wiki's FlashAttention-3 paragraph names FP8 as one of
 // FA3's Hopper features and defines nothing further.
 //
-// Two pipelines (FwdCfg::PS):
-// * P through shared memory (PS): the softmax thread reads S_t(j) out of
-//   TMEM and arrives on s_empty; the MMA issuer then starts S_t(j+1) in the
-//   same columns while block j's exponentials run.  P_t(j) goes to a K-major
-//   128-byte-swizzled shared-memory tile once P_t(j-1) V_{j-1} has released
-//   it (p_empty, which also orders the rare O~ rescale after that MMA), and
-//   P_t(j) V_j runs SMEM x SMEM.  Issue order per block: S0(j+1), S1(j+1),
-//   PV0(j), PV1(j); the producer loads K one block ahead of V.
-// * P in TMEM (kept as an option, no instance uses it now): P overwrites the
-//   upper half of S_t's columns;
-//   issue order PV0(j), S0(j+1), PV1(j), S1(j+1), so the softmax of one tile
-//   overlaps the tensor-core work of the other.  tcgen05 ops of one thread
-//   complete in issue order, and tcgen05.commit arrives after all earlier
-//   ops, so "S_t(j+1) ready" also means "PV_t(j) done": the softmax thread
-//   may rescale O~ in TMEM right then.
+// Pipeline: the softmax thread reads S_t(j) out of TMEM and arrives on
+// s_empty; the MMA issuer then starts S_t(j+1) in the same columns while
+// block j's exponentials run.  P_t(j) goes to a K-major 128-byte-swizzled
+// shared-memory tile once P_t(j-1) V_{j-1} has released it (p_empty, which
+// also orders the rare O~ rescale after that MMA), and P_t(j) V_j runs
+// SMEM x SMEM.  Issue order per block: S0(j+1), S1(j+1), PV0(j), PV1(j); the
+// producer loads K one block ahead of V.  (Keeping P in TMEM over S_t's
+// columns instead was measured slower on B200: at d = 128 the shared-memory
+// form gained 2% with a 1-stage K/V ring against 2 stages, at d = 256 with
+// one Q tile per CTA 23-35%.)
 #include <math.h>
 
 #include "common.cuh"
@@ -84,25 +79,17 @@ constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-#ifndef FA_FWD_POLY_EXP
-#define FA_FWD_POLY_EXP 0
-#endif
-// When on, one column in four of P takes its exponential from exp2_poly (FMA
-// pipe) instead of MUFU.  Off by default: on B200 it measured 3-5% slower
-// than MUFU alone, so the exponential unit is not what bounds this kernel.
-constexpr bool kPolyExp = FA_FWD_POLY_EXP != 0;
 
 // ES: bytes per Q/K/V element, 2 for bf16, 1 for e4m3.  Tiles are laid out in
 // bytes (128-byte swizzled rows), so an e4m3 d = 128 tile has the shape of a
 // bf16 d = 64 one.
-// PS: P goes to shared memory instead of TMEM, which frees S's TMEM columns
-// as soon as the softmax has read them, so S(j+1) is issued while the softmax
-// of block j still runs.
-template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2, bool PS_ = false>
+// P goes to shared memory, which frees S's TMEM columns as soon as the
+// softmax has read them, so S(j+1) is issued while the softmax of block j
+// still runs.
+template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2>
 struct FwdCfg {
   static constexpr int D = D_, NT = NT_, BN = BN_, STAGES = STAGES_, ES = ES_;
   static constexpr bool F8 = ES == 1;
-  static constexpr bool PS = PS_;
   static constexpr int DCH = D * ES / 128;                // 128-byte column chunks
   static constexpr int CH_ELEMS = 128 / ES;               // elements per chunk (TMA box width)
   static constexpr int MMA_K = 32 / ES;                   // K of one MMA: 32 bytes of a row
@@ -120,16 +107,16 @@ struct FwdCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NT * Q_TILE;
   static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
-  // P tiles (PS): [NT][BM rows][BN * ES bytes], K-major 128-byte swizzled chunks
+  // P tiles: [NT][BM rows][BN * ES bytes], K-major 128-byte swizzled chunks
   static constexpr int P_ROWB = BN * ES;
   static constexpr int P_CHUNK = BM * 128;
-  static constexpr int P_TILE = PS ? P_CHUNK * (P_ROWB / 128) : 0;
+  static constexpr int P_TILE = P_CHUNK * (P_ROWB / 128);
   static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;
   static constexpr int OFF_BAR = OFF_P + NT * P_TILE;
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NT],
-  // p_full[NT], o_full[NT], drain, q_empty, o_empty[NT]; PS adds
-  // s_empty[NT] (S read out of TMEM) and p_empty[NT] (P V done with P)
-  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NT + 1 + 1 + NT + (PS ? 2 * NT : 0);
+  // p_full[NT], o_full[NT], drain, q_empty, o_empty[NT], s_empty[NT] (S read
+  // out of TMEM), p_empty[NT] (P V done with P)
+  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NT + 1 + 1 + NT + 2 * NT;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem base slot, abort flag
   static constexpr int SMEM = OFF_MISC + 16 + 1024;       // + alignment slack
   // TMEM columns
@@ -178,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_SFULL = 1 + 4 * C::STAGES, B_PFULL = B_SFULL + C::NT, B_OFULL = B_PFULL + C::NT;
   const int B_DRAIN = B_OFULL + C::NT;
   const int B_QEMPTY = B_DRAIN + 1, B_OEMPTY = B_DRAIN + 2;
-  const int B_SEMPTY = B_OEMPTY + C::NT, B_PEMPTY = B_SEMPTY + C::NT;   // PS only
+  const int B_SEMPTY = B_OEMPTY + C::NT, B_PEMPTY = B_SEMPTY + C::NT;
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
 
@@ -229,10 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_PFULL + t), BM);
       mbar_init(bar(B_OFULL + t), 1);
       mbar_init(bar(B_OEMPTY + t), BM);
-      if constexpr (C::PS) {
-        mbar_init(bar(B_SEMPTY + t), BM);
-        mbar_init(bar(B_PEMPTY + t), 1);
-      }
+      mbar_init(bar(B_SEMPTY + t), BM);
+      mbar_init(bar(B_PEMPTY + t), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -303,19 +288,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           last_v_phase[s] = ph;
           return true;
         };
-        // Loads follow the MMA issuer's order of use: K_j, V_j, K_{j+1}, ...,
-        // or with PS (S runs a block ahead) K_0, K_1, V_0, K_2, V_1, ...
-        if constexpr (C::PS) {
-          ok = load_k(0);
-          for (int j = 0; j < U.nkb && ok; ++j) {
-            if (j + 1 < U.nkb) ok = load_k(j + 1);
-            if (ok) ok = load_v(j);
-          }
-        } else {
-          for (int j = 0; j < U.nkb && ok; ++j) {
-            ok = load_k(j);
-            if (ok) ok = load_v(j);
-          }
+        // Loads follow the MMA issuer's order of use (S runs a block ahead):
+        // K_0, K_1, V_0, K_2, V_1, ...
+        ok = load_k(0);
+        for (int j = 0; j < U.nkb && ok; ++j) {
+          if (j + 1 < U.nkb) ok = load_k(j + 1);
+          if (ok) ok = load_v(j);
         }
         g += U.nkb;
         ++uq;
@@ -356,25 +334,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dp0 = sw128_desc(sbase + C::OFF_P, 16, 1024);
     auto issue_PV = [&](int t, int s, bool first) {
       const uint64_t vb = desc_add(dv0, s * C::KV_TILE);
-      const uint32_t pcol = tmem + C::TM_S + t * C::BN + C::BN / 2;
       const uint64_t pa = desc_add(dp0, t * C::P_TILE);
 #pragma unroll
       for (int kk = 0; kk < C::PV_STEPS; ++kk) {
-        // MMA_K keys of P = 8 TMEM columns (two bf16 or four e4m3 per column),
-        // or 32 bytes of a K-major shared-memory P row (PS); MMA_K rows of the
-        // MN-major V tile
+        // 32 bytes of a K-major shared-memory P row (MMA_K keys); MMA_K rows
+        // of the MN-major V tile
         const uint32_t offp = (kk >> 2) * C::P_CHUNK + (kk & 3) * 32;
-        if constexpr (C::PS && C::F8)
+        if constexpr (C::F8)
           mma_ss_f8(tmem + C::TM_O + t * C::D, desc_add(pa, offp), desc_add(vb, kk * C::MMA_K * 128),
                     IDESC_PV, (!first) || kk > 0);
-        else if constexpr (C::PS)
-          mma_ss(tmem + C::TM_O + t * C::D, desc_add(pa, offp), desc_add(vb, kk * C::MMA_K * 128),
-                 IDESC_PV, (!first) || kk > 0);
-        else if constexpr (C::F8)
-          mma_ts_f8(tmem + C::TM_O + t * C::D, pcol + kk * 8, desc_add(vb, kk * C::MMA_K * 128),
-                    IDESC_PV, (!first) || kk > 0);
         else
-          mma_ts(tmem + C::TM_O + t * C::D, pcol + kk * 8, desc_add(vb, kk * C::MMA_K * 128),
+          mma_ss(tmem + C::TM_O + t * C::D, desc_add(pa, offp), desc_add(vb, kk * C::MMA_K * 128),
                  IDESC_PV, (!first) || kk > 0);
       }
     };
@@ -400,78 +370,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(bar(B_KEMPTY + g % C::STAGES));
         if (U.nkb == 1) mma_commit(bar(B_QEMPTY));   // last S of the unit issued
-        if constexpr (C::PS) {
-          // S_t(j+1) as soon as the softmax has read S_t(j); P_t(j) V_j once
-          // P_t(j) is in shared memory.
-          for (int j = 0; j < U.nkb && ok; ++j) {
-            const int gj = g + j;
-            const int s = gj % C::STAGES;
-            const uint32_t ph = (gj / C::STAGES) & 1;
-            if (j + 1 < U.nkb) {
-              const int s1 = (gj + 1) % C::STAGES;
-              ok = bounded_wait(bar(B_KFULL + s1), ((gj + 1) / C::STAGES) & 1, wc);
-              for (int t = 0; t < C::NT && ok; ++t) {
-                ok = bounded_wait(bar(B_SEMPTY + t), gj & 1, wc);
-                if (!ok) break;
-                tc_fence_after();
-                issue_S(t, s1);
-                mma_commit(bar(B_SFULL + t));
-              }
-              if (!ok) break;
-              mma_commit(bar(B_KEMPTY + s1));
-              if (j + 2 == U.nkb) mma_commit(bar(B_QEMPTY));   // last S of the unit
-            }
-            ok = bounded_wait(bar(B_VFULL + s), ph, wc);
-            for (int t = 0; t < C::NT && ok; ++t) {
-              ok = bounded_wait(bar(B_PFULL + t), gj & 1, wc);
-              if (ok && j == 0 && uq > 0)   // the previous unit's epilogue has read O_t
-                ok = bounded_wait(bar(B_OEMPTY + t), (uq - 1) & 1, wc);
-              if (!ok) break;
-              tc_fence_after();
-              issue_PV(t, s, j == 0);
-              mma_commit(bar(B_PEMPTY + t));
-              if (j + 1 == U.nkb) mma_commit(bar(B_OFULL + t));
-            }
-            if (ok) mma_commit(bar(B_VEMPTY + s));
-          }
-          g += U.nkb;
-          ++uq;
-          continue;
-        }
+        // S_t(j+1) as soon as the softmax has read S_t(j); P_t(j) V_j once
+        // P_t(j) is in shared memory.
         for (int j = 0; j < U.nkb && ok; ++j) {
           const int gj = g + j;
           const int s = gj % C::STAGES;
           const uint32_t ph = (gj / C::STAGES) & 1;
-          const int s1 = (gj + 1) % C::STAGES;
-          const uint32_t ph1 = ((gj + 1) / C::STAGES) & 1;
-          ok = bounded_wait(bar(B_VFULL + s), ph, wc);
-          if (!ok) break;
-          for (int t = 0; t < C::NT && ok; ++t) {
-            ok = bounded_wait(bar(B_PFULL + t), gj & 1, wc);
-            if (!ok) break;
-            if (t == 0 && j + 1 < U.nkb) {
-              ok = bounded_wait(bar(B_KFULL + s1), ph1, wc);
+          if (j + 1 < U.nkb) {
+            const int s1 = (gj + 1) % C::STAGES;
+            ok = bounded_wait(bar(B_KFULL + s1), ((gj + 1) / C::STAGES) & 1, wc);
+            for (int t = 0; t < C::NT && ok; ++t) {
+              ok = bounded_wait(bar(B_SEMPTY + t), gj & 1, wc);
               if (!ok) break;
-            }
-            if (j == 0 && uq > 0) {
-              // the previous unit's epilogue must have read O_t out of TMEM
-              ok = bounded_wait(bar(B_OEMPTY + t), (uq - 1) & 1, wc);
-              if (!ok) break;
-            }
-            tc_fence_after();
-            issue_PV(t, s, j == 0);
-            if (j + 1 < U.nkb) {
+              tc_fence_after();
               issue_S(t, s1);
               mma_commit(bar(B_SFULL + t));
-              if (t == C::NT - 1) {
-                mma_commit(bar(B_KEMPTY + s1));
-                if (j + 2 == U.nkb) mma_commit(bar(B_QEMPTY));   // last S of the unit
-              }
-            } else {
-              mma_commit(bar(B_OFULL + t));
             }
-            if (t == C::NT - 1) mma_commit(bar(B_VEMPTY + s));
+            if (!ok) break;
+            mma_commit(bar(B_KEMPTY + s1));
+            if (j + 2 == U.nkb) mma_commit(bar(B_QEMPTY));   // last S of the unit
           }
+          ok = bounded_wait(bar(B_VFULL + s), ph, wc);
+          for (int t = 0; t < C::NT && ok; ++t) {
+            ok = bounded_wait(bar(B_PFULL + t), gj & 1, wc);
+            if (ok && j == 0 && uq > 0)   // the previous unit's epilogue has read O_t
+              ok = bounded_wait(bar(B_OEMPTY + t), (uq - 1) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            issue_PV(t, s, j == 0);
+            mma_commit(bar(B_PEMPTY + t));
+            if (j + 1 == U.nkb) mma_commit(bar(B_OFULL + t));
+          }
+          if (ok) mma_commit(bar(B_VEMPTY + s));
         }
         g += U.nkb;
         ++uq;
@@ -489,7 +419,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = threadIdx.x & 127;          // row within the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::TM_S + t * C::BN;
-    const uint32_t tP = tS + C::BN / 2;
     const uint32_t tO = tmem + lane_off + C::TM_O + t * C::D;
     bool ok = true;
     int g = 0, uq = 0;
@@ -525,11 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < C::BN / 32; ++c)
           tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_wait_ld();
-        if constexpr (C::PS) {
-          // S_t is in registers: its TMEM columns may take S_t(j+1)
-          tc_fence_before();
-          mbar_arrive(bar(B_SEMPTY + t));
-        }
+        // S_t is in registers: its TMEM columns may take S_t(j+1)
+        tc_fence_before();
+        mbar_arrive(bar(B_SEMPTY + t));
         float *s = reinterpret_cast<float *>(sr);
         const int col_lo = (U.j0 + j) * C::BN;
         const bool need_mask =
@@ -560,16 +487,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_run = m_new;
         }
         const float m_use = ((m_run == -INFINITY) ? 0.f : m_run) - C::P_SHIFT;
-        // p = 2^(s * scale * log2e - m) on MUFU (exp2_poly for one column in
-        // four when FA_FWD_POLY_EXP is set); row sum in four independent
-        // partials over the undropped p; with dropout, P in TMEM keeps only the
-        // columns whose Philox word is >= drop_thr (one Philox call per four
-        // key columns)
+        // p = 2^(s * scale * log2e - m) on MUFU; row sum in four independent
+        // partials over the undropped p; with dropout, the stored P keeps
+        // only the columns whose Philox word is >= drop_thr (one Philox call
+        // per four key columns)
         float rs[4] = {0.f, 0.f, 0.f, 0.f};
-        // PS: row r of the K-major shared-memory P tile (16-byte units
-        // swizzled by r mod 8); written chunk by chunk once P_t(j-1) V_{j-1}
-        // is done with it (waited before the first store: by then the MMA
-        // has had the row maximum and 32 exponentials' time)
+        // row r of the K-major shared-memory P tile (16-byte units swizzled
+        // by r mod 8); written chunk by chunk once P_t(j-1) V_{j-1} is done
+        // with it (waited before the first store: by then the MMA has had the
+        // row maximum and 32 exponentials' time)
         const uint32_t prow = sbase + C::OFF_P + t * C::P_TILE + r * 128;
         const int r7 = r & 7;
   #pragma unroll
@@ -581,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float x0 = fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_use);
             const float x1 = fmaf(s[c * 32 + 2 * e + 1], p.scale_log2, -m_use);
             const float p0 = fast_exp2(x0);
-            const float p1 = (kPolyExp && (e & 1)) ? exp2_poly(x1) : fast_exp2(x1);
+            const float p1 = fast_exp2(x1);
             rs[e & 3] += p0 + p1;
             if (DROP) {
               if ((e & 1) == 0)
@@ -590,42 +516,34 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t w0 = (e & 1) ? rnd.z : rnd.x, w1 = (e & 1) ? rnd.w : rnd.y;
               pk[e] = pack_bf16x2(w0 >= p.drop_thr ? p0 : 0.f, w1 >= p.drop_thr ? p1 : 0.f);
             } else if constexpr (C::F8) {
-              // four e4m3 codes per column: keys 2e, 2e + 1 in the low half
-              // of word e / 2 for even e, in the high half for odd e
+              // four e4m3 codes per 32-bit word: keys 2e, 2e + 1 in the low
+              // half of word e / 2 for even e, in the high half for odd e
               const uint32_t h = pack_e4m3x2(p0, p1);
               pk[e >> 1] = (e & 1) ? (pk[e >> 1] | (h << 16)) : h;
             } else {
               pk[e] = pack_bf16x2(p0, p1);
             }
           }
-          if constexpr (C::PS) {
-            if (c == 0 && j > 0) {
-              ok = warp_wait_all(bar(B_PEMPTY + t), (g + j - 1) & 1, wc);
-              tc_fence_after();
-            }
-            if (ok) {
+          if (c == 0 && j > 0) {
+            ok = warp_wait_all(bar(B_PEMPTY + t), (g + j - 1) & 1, wc);
+            tc_fence_after();
+          }
+          if (ok) {
   #pragma unroll
-              for (int i = 0; i < 2 * C::ES; ++i) {   // 32 keys = 2 * ES 16-byte units
-                const int b = c * 32 * C::ES + 16 * i;
-                const int u = (b >> 4) & 7;
-                st_shared_v4(prow + (b >> 7) * C::P_CHUNK + ((u ^ r7) << 4), pk[4 * i], pk[4 * i + 1],
-                             pk[4 * i + 2], pk[4 * i + 3]);
-              }
+            for (int i = 0; i < 2 * C::ES; ++i) {   // 32 keys = 2 * ES 16-byte units
+              const int b = c * 32 * C::ES + 16 * i;
+              const int u = (b >> 4) & 7;
+              st_shared_v4(prow + (b >> 7) * C::P_CHUNK + ((u ^ r7) << 4), pk[4 * i], pk[4 * i + 1],
+                           pk[4 * i + 2], pk[4 * i + 3]);
             }
-          } else if constexpr (C::F8) {
-            tmem_st8(tP + c * 8, *reinterpret_cast<const uint32_t(*)[8]>(pk));
-          } else {
-            tmem_st16(tP + c * 16, pk);
           }
         }
         const float rowsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
         l_run = l_run * alpha + rowsum;
-        if constexpr (C::PS) {
-          if (!ok) break;
-          fence_proxy_async_smem();   // P stores visible to the tensor core
-        }
-        // (PS: P_t(j-1) V_{j-1}, which accumulates into O_t, was waited for
-        // above, so O_t may be rescaled)
+        if (!ok) break;
+        fence_proxy_async_smem();   // P stores visible to the tensor core
+        // (P_t(j-1) V_{j-1}, which accumulates into O_t, was waited for above,
+        // so O_t may be rescaled)
         if (rescale) {
   #pragma unroll 1
           for (int c = 0; c < C::D / 32; ++c) {
@@ -878,17 +796,17 @@ int launch_fwd_splitkv_bf16_sm100(const AttnArgs &a) {
 
 int launch_fwd_e4m3_sm100(const AttnArgs &a) {
   switch (a.d) {
-    case 128: return run_fwd<FwdCfg<128, 2, 128, 3, 1, true>>(a);
-    case 256: return run_fwd<FwdCfg<256, 1, 128, 2, 1, true>>(a);
+    case 128: return run_fwd<FwdCfg<128, 2, 128, 3, 1>>(a);
+    case 256: return run_fwd<FwdCfg<256, 1, 128, 2, 1>>(a);
     default: return 2;
   }
 }
 
 int launch_fwd_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {
-    case 64: return run_fwd<FwdCfg<64, 2, 128, 3, 2, true>>(a);
-    case 128: return run_fwd<FwdCfg<128, 2, 128, 1, 2, true>>(a);
-    case 256: return run_fwd<FwdCfg<256, 1, 128, 1, 2, true>>(a);
+    case 64: return run_fwd<FwdCfg<64, 2, 128, 3, 2>>(a);
+    case 128: return run_fwd<FwdCfg<128, 2, 128, 1, 2>>(a);
+    case 256: return run_fwd<FwdCfg<256, 1, 128, 1, 2>>(a);
     default: return 2;
   }
 }

@@ -75,7 +75,6 @@ int launch_bwd_prep_bf16(const AttnArgs &a);     // D + zeroed dQ accumulator
 int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a);
 int launch_bwd_dq_bf16(const AttnArgs &a);       // dq = bf16(scale * accumulator)
 int launch_wait_selftest(long long timeout_ns, cudaStream_t stream, unsigned *err);
-int launch_exp2_eval(const float *x, float *y, int n, int poly, cudaStream_t stream);
 
 // Argument checks and per-call device set-up shared by the C entry points
 // (fa_status codes): size/scale rules, then current device, architecture and

@@ -273,15 +273,6 @@ int fa_device_status(fa_stream_t stream);
  */
 int fa_wait_selftest(long long timeout_ns, fa_stream_t stream);
 
-/*
- * fa_exp2_eval -- y[i] = 2^x[i] for n device floats, with the exponential the
- * softmax kernels use: poly != 0 selects the FMA-pipe polynomial (range
- * reduction to [-1/2, 1/2] and a fitted cubic, exact at integers, relative
- * error < 1.1e-4 for -126 <= x <= 127), poly == 0 the hardware ex2.approx.  Exists so tests can
- * bound the polynomial's error.
- */
-int fa_exp2_eval(const float *x, float *y, int n, int poly, fa_stream_t stream);
-
 /* fa_strerror -- static description of a status code. */
 const char *fa_strerror(int status);
 

@@ -155,36 +155,3 @@ def test_bf16_backward_repeatable_within_tolerance():
         rel = float((a.float() - b.float()).norm() / b.float().norm())
         assert rel < 1e-3
     assert torch.equal(r1[1], r2[1]) and torch.equal(r1[2], r2[2])  # dK, dV deterministic
-
-
-# ------------------------------------------------------- polynomial exp2
-def test_exp2_polynomial_error_bound():
-    """The FMA-pipe 2^x used for part of the softmax stays within 1.1e-4
-    relative error of the exact value on [-126, 127] (the fitted cubic's bound
-    is 1.02e-4), is exact at integers, and agrees with the hardware ex2 to the
-    same bound; masked inputs (-inf) give ~0."""
-    g = torch.Generator().manual_seed(5)
-    x = torch.cat([torch.rand(200000, generator=g, dtype=torch.float64) * 40 - 32,
-                   torch.rand(20000, generator=g, dtype=torch.float64) * 253 - 126,
-                   torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 8.0, -126.0, 127.0, -125.5])]).float()
-    xd = x.cuda()
-    yp = torch.empty_like(xd)
-    yh = torch.empty_like(xd)
-    assert F.fa_exp2_eval(xd.data_ptr(), yp.data_ptr(), x.numel(), 1) == F.FA_OK
-    assert F.fa_exp2_eval(xd.data_ptr(), yh.data_ptr(), x.numel(), 0) == F.FA_OK
-    torch.cuda.synchronize()
-    exact = torch.exp2(x.double())
-    rel_p = ((yp.cpu().double() - exact).abs() / exact).max().item()
-    rel_h = ((yp.cpu().double() - yh.cpu().double()).abs() / exact).max().item()
-    assert rel_p < 1.1e-4, rel_p
-    assert rel_h < 1.2e-4, rel_h
-    ints = torch.arange(-126, 128, dtype=torch.float32, device="cuda")
-    yi = torch.empty_like(ints)
-    assert F.fa_exp2_eval(ints.data_ptr(), yi.data_ptr(), ints.numel(), 1) == F.FA_OK
-    torch.cuda.synchronize()
-    assert torch.equal(yi.cpu().double(), torch.exp2(ints.cpu().double()))
-    z = torch.tensor([float("-inf"), -300.0, -127.0], device="cuda")
-    yz = torch.empty_like(z)
-    assert F.fa_exp2_eval(z.data_ptr(), yz.data_ptr(), 3, 1) == F.FA_OK
-    torch.cuda.synchronize()
-    assert bool((yz >= 0).all()) and float(yz.max()) < 2.0 ** -124
