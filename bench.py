@@ -71,6 +71,13 @@ def measured_peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+def peak_label(src, what="bf16 dense burst"):
+    """Where the roofline denominator came from."""
+    if src == "measured":
+        return f"measured {what} (MEASURED_PEAKS.json)"
+    return f"fallback {what} (no MEASURED_PEAKS.json on this machine)"
+
+
 def l2_note(w):
     """How the GPU arm keeps the timed inputs out of L2 (126 MB) for this
     workload: inputs larger than L2, or otherwise what stays resident."""
@@ -327,7 +334,7 @@ def run_ours(args, rank, world, local_rank):
         "bwd_tflops": round(bwd_f / ((mean["prep"] + mean["dkdv"] + mean["dq"]) * 1e-3) / 1e12, 2),
         "roofline": {"bound": "tensor", "kernel": "fa_fwd" if dom == "fwd" else "fa_bwd_dkdv",
                      "achieved": round(achieved, 2), "peak": burst,
-                     "peak_source": f"{src} bf16 dense burst (MEASURED_PEAKS.json)",
+                     "peak_source": peak_label(src),
                      "unit": "TFLOP/s", "frac": round(achieved / burst, 4), "traffic": traffic},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
@@ -514,12 +521,12 @@ def run_forward_only(args, rank, world, local_rank):
     if fp8:
         # e4m3 dense peak: the measured bf16 burst times the nominal ratio
         # (4.5 / 2.25 PFLOP/s dense)
-        peak, peak_src = 2.0 * burst, f"{src} bf16 dense burst x 2 (nominal e4m3/bf16 ratio)"
+        peak, peak_src = 2.0 * burst, peak_label(src, "bf16 dense burst x 2 (nominal e4m3/bf16 ratio)")
         metric = METRIC_FP8
         data = "synthetic (seeded N(0,1) float32 quantised per tensor to e4m3, shapes of the workload)"
         kernel = "fa_fwd_fp8"
     else:
-        peak, peak_src = burst, f"{src} bf16 dense burst (MEASURED_PEAKS.json)"
+        peak, peak_src = burst, peak_label(src)
         metric = METRIC_SPLITKV
         data = "synthetic (seeded N(0,1) bf16, shapes of the workload)"
         kernel = "fa_fwd_splitkv (pieces + merge)"
