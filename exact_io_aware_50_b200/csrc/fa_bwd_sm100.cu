@@ -108,8 +108,8 @@ struct BwdCfg {
   static constexpr int OFF_DD = OFF_L2 + QS * ROWVEC;
   static constexpr int OFF_BAR = OFF_DD + QS * ROWVEC;
   // kv_full, kc_full, q_full[QS], q_empty[QS], s_full[2], p_full[2],
-  // dq_full[2], dq_empty[2], final, drain
-  static constexpr int NBAR = 2 + 2 * QS + 8 + 2;
+  // dq_full[2], dq_empty[2], final, drain, do_full[QS], do_empty[QS]
+  static constexpr int NBAR = 2 + 2 * QS + 8 + 2 + 2 * QS;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
   // so no alignment slack is reserved.
@@ -220,7 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return smem_u32(bars + i); };
   const int B_KV = 0, B_KC = 1, B_QFULL = 2, B_QEMPTY = 2 + C::QS, B_SFULL = 2 + 2 * C::QS,
             B_PFULL = B_SFULL + 2, B_DQFULL = B_PFULL + 2, B_DQEMPTY = B_DQFULL + 2,
-            B_FINAL = B_DQEMPTY + 2, B_DRAIN = B_FINAL + 1;
+            B_FINAL = B_DQEMPTY + 2, B_DRAIN = B_FINAL + 1, B_DOFULL = B_DRAIN + 1,
+            B_DOEMPTY = B_DOFULL + C::QS;
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
   const float *s_l2 = (const float *)(smem + C::OFF_L2);
@@ -252,6 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::QS; ++s) {
       mbar_init(bar(B_QFULL + s), 1);
       mbar_init(bar(B_QEMPTY + s), 1);
+      mbar_init(bar(B_DOFULL + s), 1);
+      mbar_init(bar(B_DOEMPTY + s), 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(B_SFULL + x), 1);
@@ -284,8 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     // The whole role runs in lane 0; the other lanes wait at the end.
     if (lane == 0) {
-      int last_phase[C::QS];
-      for (int s = 0; s < C::QS; ++s) last_phase[s] = -1;
+      int last_q[C::QS], last_do[C::QS];
+      for (int s = 0; s < C::QS; ++s) last_q[s] = last_do[s] = -1;
       bool ok = true;
       mbar_arrive_expect_tx(bar(B_KV), (C::HAS_DP ? 2 : 1) * C::KV_TILE);
       for (int c = 0; c < C::DCH; ++c) {
@@ -293,32 +296,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (C::HAS_DP)
           tma_load_3d(sbase + C::OFF_V + c * C::KV_CHUNK, &tmV, bar(B_KV), c * 64, kv0, bhkv);
       }
+      // Q_i with the row vectors L2_i, D_i (read by S^T, dK and the
+      // elementwise stage) and dO_i (read only by dP^T in the dK/dQ pass, by
+      // dV in the dV pass) fill separate slots, so dO_{i+1} can arrive as soon
+      // as dP^T(i) is done and Q_{i+1} as soon as dK(i) is.
+      auto load_q = [&](int i, int st, uint32_t ph) {
+        if (!bounded_wait(bar(B_QEMPTY + st), ph ^ 1, wc)) return false;
+        const int h = step_head(i), qb = step_qblk(i);
+        const int bh = b * p.Hq + h;
+        const size_t vrow = (size_t)bh * p.npad + (size_t)qb * C::BM;
+        const uint32_t fb = bar(B_QFULL + st);
+        mbar_arrive_expect_tx(fb, C::Q_TILE + 2 * C::ROWVEC);
+        for (int c = 0; c < C::DCH; ++c)
+          tma_load_3d(sbase + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, fb, c * 64,
+                      qb * C::BM, bh);
+        bulk_load(sbase + C::OFF_L2 + st * C::ROWVEC, p.l2 + vrow, C::ROWVEC, fb);
+        bulk_load(sbase + C::OFF_DD + st * C::ROWVEC, p.dsum + vrow, C::ROWVEC, fb);
+        last_q[st] = ph;
+        return true;
+      };
+      auto load_do = [&](int i, int st, uint32_t ph) {
+        if (!bounded_wait(bar(B_DOEMPTY + st), ph ^ 1, wc)) return false;
+        const int bh = b * p.Hq + step_head(i), qb = step_qblk(i);
+        const uint32_t fb = bar(B_DOFULL + st);
+        mbar_arrive_expect_tx(fb, C::Q_TILE);
+        for (int c = 0; c < C::DCH; ++c)
+          tma_load_3d(sbase + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmDO, fb, c * 64,
+                      qb * C::BM, bh);
+        last_do[st] = ph;
+        return true;
+      };
       for (int i = 0; i < nsteps && ok; ++i) {
         const int st = i % C::QS;
         const uint32_t ph = (i / C::QS) & 1;
-        ok = bounded_wait(bar(B_QEMPTY + st), ph ^ 1, wc);
-        if (!ok) break;
-        {
-          const int h = step_head(i), qb = step_qblk(i);
-          const int bh = b * p.Hq + h;
-          const size_t vrow = (size_t)bh * p.npad + (size_t)qb * C::BM;
-          const uint32_t fb = bar(B_QFULL + st);
-          mbar_arrive_expect_tx(fb, 2 * C::Q_TILE + 2 * C::ROWVEC);
-          for (int c = 0; c < C::DCH; ++c) {
-            tma_load_3d(sbase + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, fb, c * 64,
-                        qb * C::BM, bh);
-            tma_load_3d(sbase + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmDO, fb, c * 64,
-                        qb * C::BM, bh);
-          }
-          bulk_load(sbase + C::OFF_L2 + st * C::ROWVEC, p.l2 + vrow, C::ROWVEC, fb);
-          bulk_load(sbase + C::OFF_DD + st * C::ROWVEC, p.dsum + vrow, C::ROWVEC, fb);
+        // the slot freed first goes first: dO in the dK/dQ pass, Q in the dV pass
+        if (C::HAS_DP) {
+          ok = load_do(i, st, ph);
+          if (ok) ok = load_q(i, st, ph);
+        } else {
+          ok = load_q(i, st, ph);
+          if (ok) ok = load_do(i, st, ph);
         }
-        last_phase[st] = ph;
       }
       if (!ok) {
         (void)drain_wait(bar(B_KV), 0, p.err, kWaitLimitNs);
-        for (int s = 0; s < C::QS; ++s)
-          if (last_phase[s] >= 0) (void)drain_wait(bar(B_QFULL + s), last_phase[s], p.err, kWaitLimitNs);
+        for (int s = 0; s < C::QS; ++s) {
+          if (last_q[s] >= 0) (void)drain_wait(bar(B_QFULL + s), last_q[s], p.err, kWaitLimitNs);
+          if (last_do[s] >= 0) (void)drain_wait(bar(B_DOFULL + s), last_do[s], p.err, kWaitLimitNs);
+        }
       }
     }
     __syncwarp();
@@ -394,6 +419,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                  IDESC_DQ, kk > 0);
       }
     };
+    // S^T(i) (and dP^T(i) in the dK/dQ pass) into score set x.  The caller
+    // has waited for Q_i; dO_i is waited for here and its slot released once
+    // dP^T(i) is done with it.
+    auto issue_scores = [&](int x, int i) {
+      const int st = i % C::QS;
+      issue_S(x, st);
+      if (C::HAS_DP) {
+        if (!bounded_wait(bar(B_DOFULL + st), (i / C::QS) & 1, wc)) return false;
+        tc_fence_after();
+        issue_dP(x, st);
+        mma_commit(bar(B_DOEMPTY + st));
+      }
+      mma_commit(bar(B_SFULL + x));
+      return true;
+    };
     // The whole role runs in lane 0; the other lanes wait at the end.
     if (lane == 0) {
     // K - c must be in place before the first MMA reads K
@@ -402,11 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = bounded_wait(bar(B_QFULL + 0), 0, wc);
       if (ok) {
         tc_fence_after();
-        {
-          issue_S(0, 0);
-          issue_dP(0, 0);
-          mma_commit(bar(B_SFULL + 0));
-        }
+        ok = issue_scores(0, 0);
       }
     }
     for (int i = 0; i < nsteps && ok; ++i) {
@@ -422,11 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = bounded_wait(bar(B_QFULL + st1), ((i + 1) / C::QS) & 1, wc);
         if (!ok) break;
         tc_fence_after();
-        {
-          issue_S(y, st1);
-          issue_dP(y, st1);
-          mma_commit(bar(B_SFULL + y));
-        }
+        ok = issue_scores(y, i + 1);
+        if (!ok) break;
       }
       ok = bounded_wait(bar(B_PFULL + x), set_phase(i), wc);
       if (!ok) break;
@@ -434,27 +467,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = bounded_wait(bar(B_DQEMPTY + x), set_phase(i - 1), wc);
         if (!ok) break;
       }
+      if (!C::HAS_DP) {
+        // the dV pass reads dO_i in dV(i)
+        ok = bounded_wait(bar(B_DOFULL + st), (i / C::QS) & 1, wc);
+        if (!ok) break;
+      }
       tc_fence_after();
-      {
-        issue_dvdk(x, st, i == 0);
-        if (C::HAS_DQ) {
-          issue_dq(x);
-          mma_commit(bar(B_DQFULL + x));
-        }
-        mma_commit(bar(B_QEMPTY + st));
+      issue_dvdk(x, st, i == 0);
+      // Q_i is done with once dK(i) (or S^T(i) in the dV pass) has read it;
+      // the elementwise stage finished with L2_i and D_i before p_full.  dQ^T(i)
+      // reads K and dS^T only.
+      mma_commit(bar(B_QEMPTY + st));
+      if (!C::HAS_DP) mma_commit(bar(B_DOEMPTY + st));
+      if (C::HAS_DQ) {
+        issue_dq(x);
+        mma_commit(bar(B_DQFULL + x));
       }
       if (C::NSETS == 1 && i + 1 < nsteps) {
         // S^T(i+1) only overwrites P^T/dS^T, which dV/dK(i) (issued earlier)
-        // consume in order
+        // consume in order; Q_{i+1} arrives while dQ^T(i) runs
         const int st1 = (i + 1) % C::QS;
         ok = bounded_wait(bar(B_QFULL + st1), ((i + 1) / C::QS) & 1, wc);
         if (!ok) break;
         tc_fence_after();
-        issue_S(x, st1);
-        {
-          issue_dP(x, st1);
-          mma_commit(bar(B_SFULL + x));
-        }
+        ok = issue_scores(x, i + 1);
+        if (!ok) break;
       }
     }
     if (ok) {
