@@ -296,22 +296,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (C::HAS_DP)
           tma_load_3d(sbase + C::OFF_V + c * C::KV_CHUNK, &tmV, bar(B_KV), c * 64, kv0, bhkv);
       }
-      // Q_i with the row vectors L2_i, D_i (read by S^T, dK and the
-      // elementwise stage) and dO_i (read only by dP^T in the dK/dQ pass, by
-      // dV in the dV pass) fill separate slots, so dO_{i+1} can arrive as soon
-      // as dP^T(i) is done and Q_{i+1} as soon as dK(i) is.
+      // Q_i and dO_i fill separate slots.  dK/dQ pass: Q_i carries the row
+      // vectors L2_i, D_i (read by the elementwise stage, Q_i last read by
+      // dK(i)) and dO_i is read only by dP^T(i), so dO_{i+1} can arrive as soon
+      // as dP^T(i) is done and Q_{i+1} as soon as dK(i) is.  dV pass: Q_i is
+      // read only by S^T(i) and the row vectors travel with dO_i (read by
+      // dV(i)), so Q_{i+2} can arrive while step i's elementwise work runs.
+      constexpr uint32_t ROWS_Q = C::HAS_DP ? 2 * C::ROWVEC : 0;
+      constexpr uint32_t ROWS_DO = C::HAS_DP ? 0 : 2 * C::ROWVEC;
+      auto load_rows = [&](int i, int st, uint32_t fb) {
+        const int bh = b * p.Hq + step_head(i);
+        const size_t vrow = (size_t)bh * p.npad + (size_t)step_qblk(i) * C::BM;
+        bulk_load(sbase + C::OFF_L2 + st * C::ROWVEC, p.l2 + vrow, C::ROWVEC, fb);
+        bulk_load(sbase + C::OFF_DD + st * C::ROWVEC, p.dsum + vrow, C::ROWVEC, fb);
+      };
       auto load_q = [&](int i, int st, uint32_t ph) {
         if (!bounded_wait(bar(B_QEMPTY + st), ph ^ 1, wc)) return false;
-        const int h = step_head(i), qb = step_qblk(i);
-        const int bh = b * p.Hq + h;
-        const size_t vrow = (size_t)bh * p.npad + (size_t)qb * C::BM;
+        const int bh = b * p.Hq + step_head(i), qb = step_qblk(i);
         const uint32_t fb = bar(B_QFULL + st);
-        mbar_arrive_expect_tx(fb, C::Q_TILE + 2 * C::ROWVEC);
+        mbar_arrive_expect_tx(fb, C::Q_TILE + ROWS_Q);
         for (int c = 0; c < C::DCH; ++c)
           tma_load_3d(sbase + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, fb, c * 64,
                       qb * C::BM, bh);
-        bulk_load(sbase + C::OFF_L2 + st * C::ROWVEC, p.l2 + vrow, C::ROWVEC, fb);
-        bulk_load(sbase + C::OFF_DD + st * C::ROWVEC, p.dsum + vrow, C::ROWVEC, fb);
+        if (ROWS_Q) load_rows(i, st, fb);
         last_q[st] = ph;
         return true;
       };
@@ -319,10 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!bounded_wait(bar(B_DOEMPTY + st), ph ^ 1, wc)) return false;
         const int bh = b * p.Hq + step_head(i), qb = step_qblk(i);
         const uint32_t fb = bar(B_DOFULL + st);
-        mbar_arrive_expect_tx(fb, C::Q_TILE);
+        mbar_arrive_expect_tx(fb, C::Q_TILE + ROWS_DO);
         for (int c = 0; c < C::DCH; ++c)
           tma_load_3d(sbase + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmDO, fb, c * 64,
                       qb * C::BM, bh);
+        if (ROWS_DO) load_rows(i, st, fb);
         last_do[st] = ph;
         return true;
       };
@@ -420,11 +428,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     // S^T(i) (and dP^T(i) in the dK/dQ pass) into score set x.  The caller
-    // has waited for Q_i; dO_i is waited for here and its slot released once
-    // dP^T(i) is done with it.
+    // has waited for Q_i; in the dV pass Q_i's slot is released once S^T(i)
+    // is done with it.  dO_i is waited for here and, in the dK/dQ pass, its
+    // slot released once dP^T(i) is done with it.
     auto issue_scores = [&](int x, int i) {
       const int st = i % C::QS;
       issue_S(x, st);
+      if (!C::HAS_DP) mma_commit(bar(B_QEMPTY + st));
       if (C::HAS_DP) {
         if (!bounded_wait(bar(B_DOFULL + st), (i / C::QS) & 1, wc)) return false;
         tc_fence_after();
@@ -474,11 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       issue_dvdk(x, st, i == 0);
-      // Q_i is done with once dK(i) (or S^T(i) in the dV pass) has read it;
-      // the elementwise stage finished with L2_i and D_i before p_full.  dQ^T(i)
-      // reads K and dS^T only.
-      mma_commit(bar(B_QEMPTY + st));
-      if (!C::HAS_DP) mma_commit(bar(B_DOEMPTY + st));
+      // dK/dQ pass: Q_i is done with once dK(i) has read it, and the
+      // elementwise stage finished with L2_i and D_i before p_full; dQ^T(i)
+      // reads K and dS^T only.  dV pass: dO_i and its row vectors likewise.
+      mma_commit(bar(C::HAS_DP ? B_QEMPTY + st : B_DOEMPTY + st));
       if (C::HAS_DQ) {
         issue_dq(x);
         mma_commit(bar(B_DQFULL + x));
@@ -543,7 +552,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int NCB = C::BM / 64;   // 32-column blocks per warpgroup and step
     for (int i = 0; i < nsteps && ok; ++i) {
       const int x = set_of(i), st = i % C::QS;
-      ok = warp_wait_all(bar(B_QFULL + st), (i / C::QS) & 1, wc);
+      // the row vectors L2_i, D_i come with Q_i (dK/dQ pass) or dO_i (dV pass)
+      ok = warp_wait_all(bar((C::HAS_DP ? B_QFULL : B_DOFULL) + st), (i / C::QS) & 1, wc);
       if (ok) ok = warp_wait_all(bar(B_SFULL + x), set_phase(i), wc);
       if (!ok) break;
       tc_fence_after();
