@@ -772,10 +772,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // into the accumulator), 16 TMA producer, 17 MMA issuer (both in lane 0).
 // EARLY_S_: the step order that issues S^T(i+1) right after dV(i) and takes
 // dK's A operand (dS^T) from shared memory (see the comment block above).
-template <int D_, int QS_, bool EARLY_S_>
+// MASKGEN_ (the dropout instances): the readout warps, which wait most of a
+// step, evaluate the Philox words of the dropout mask two steps ahead into a
+// double-buffered bit array in shared memory (one bit per key row and query
+// column, 2 KB a step), so the elementwise stage reads 64 bits instead of
+// evaluating 16 Philox calls per step on the critical path.
+template <int D_, int QS_, bool EARLY_S_, bool MASKGEN_ = false>
 struct BwdWideCfg {
   static constexpr int D = D_, QS = QS_;
   static constexpr bool EARLY_S = EARLY_S_;
+  static constexpr bool MASKGEN = MASKGEN_;
   static constexpr int BN = 128, BM = 128;
   static constexpr int DCH = D / 64;
   static constexpr int KV_CHUNK = BN * 128;
@@ -792,10 +798,13 @@ struct BwdWideCfg {
   static constexpr int OFF_DS = OFF_DO + QS * Q_TILE;
   static constexpr int OFF_L2 = OFF_DS + DS_TILE;
   static constexpr int OFF_DD = OFF_L2 + QS * ROWVEC;
-  static constexpr int OFF_BAR = OFF_DD + QS * ROWVEC;
+  static constexpr int OFF_MASK = OFF_DD + QS * ROWVEC;   // [2][128 key rows][128 query bits]
+  static constexpr int MASK_BUF = BN * BM / 8;
+  static constexpr int OFF_BAR = OFF_MASK + (MASKGEN ? 2 * MASK_BUF : 0);
   // kv, kc, q_full[QS], q_empty[QS], s_full, dp_full, p_full, ds_full,
-  // dq_full, dq_empty, final, drain, acc_empty, unit_full[4], unit_empty[4]
-  static constexpr int NBAR = 2 + 2 * QS + 9 + 8;
+  // dq_full, dq_empty, final, drain, acc_empty, unit_full[4], unit_empty[4],
+  // mask_full[2], mask_empty[2]
+  static constexpr int NBAR = 2 + 2 * QS + 9 + 8 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;   // tmem slot, abort flag, unit queue[4]
   static constexpr int SMEM = OFF_MISC + 32;
   static constexpr int TM_DV = 0, TM_DK = D, TM_A = 2 * D, TM_B = 2 * D + 128;
@@ -826,7 +835,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             B_DPFULL = B_SFULL + 1, B_PFULL = B_SFULL + 2, B_DSFULL = B_SFULL + 3,
             B_DQFULL = B_SFULL + 4, B_DQEMPTY = B_SFULL + 5, B_FINAL = B_SFULL + 6,
             B_DRAIN = B_SFULL + 7, B_ACCEMPTY = B_SFULL + 8, B_UFULL = B_SFULL + 9,
-            B_UEMPTY = B_UFULL + 4;
+            B_UEMPTY = B_UFULL + 4, B_MFULL = B_UEMPTY + 4, B_MEMPTY = B_MFULL + 2;
+  static_assert(DROP == C::MASKGEN, "dropout instances take their mask from the readout warps");
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
   volatile int *s_queue = (volatile int *)(smem + C::OFF_MISC + 16);   // unit of the k-th turn, k % 4
@@ -890,6 +900,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int s = 0; s < 4; ++s) {
       mbar_init(bar(B_UFULL + s), 1);
       mbar_init(bar(B_UEMPTY + s), 17);   // MMA issuer + 8 elementwise + 8 readout warps
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_MFULL + s), 256);    // the readout threads wrote their mask bits
+      mbar_init(bar(B_MEMPTY + s), 256);   // the elementwise threads read theirs
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -1218,7 +1232,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ---- phase 1: P^T for query columns [64 wg, 64 wg + 64), 16 at a time
         uint32_t pkeep[4][8];
         uint32_t keepbits[2] = {0u, 0u};               // dropout: bit c = column 64 wg + c kept
-        const uint32_t bhq = (uint32_t)(U.b * p.Hq + step_head(U, i));
+        if (DROP) {
+          ok = warp_wait_all(bar(B_MFULL + (gi & 1)), (gi >> 1) & 1, wc);
+          if (!ok) break;
+          const uint2 kb = *reinterpret_cast<const uint2 *>(smem + C::OFF_MASK + (gi & 1) * C::MASK_BUF +
+                                                            r * (C::BM / 8) + 8 * wg);
+          keepbits[0] = kb.x;
+          keepbits[1] = kb.y;
+          mbar_arrive(bar(B_MEMPTY + (gi & 1)));
+        }
 #pragma unroll
         for (int sb = 0; sb < 4; ++sb) {
           const int c0 = 64 * wg + 16 * sb;
@@ -1248,11 +1270,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           // all of which this thread has already read.  With dropout the dV
           // operand is P^T * Z; pkeep keeps P^T for dS.
           if (DROP) {
-            uint32_t m16 = 0;
-#pragma unroll
-            for (int gq = 0; gq < 4; ++gq)
-              m16 |= dropout_keep4(kv, q0 + c0 + 4 * gq, bhq, p, lane) << (4 * gq);
-            keepbits[sb >> 1] |= m16 << (16 * (sb & 1));
+            const uint32_t m16 = (keepbits[sb >> 1] >> (16 * (sb & 1))) & 0xffffu;
             uint32_t pm[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -1356,39 +1374,135 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t src = tmem + ((uint32_t)(quad * 32) << 16) + C::TM_B + ch0 * 32;
     const bool live_rows = quad * 32 < C::D;    // d = 64: lanes 64..127 carry no dQ
     bool ok = true;
-    int gs = 0;
-    for (int k = 0; ok; ++k) {
-      ok = warp_wait_all(bar(B_UFULL + (k & 3)), (k >> 2) & 1, wc);
-      if (!ok) break;
-      const int u = s_queue[k & 3];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_UEMPTY + (k & 3)));
-      if (u < 0) break;
-      const Unit U = decode(u);
-      for (int i = 0; i < U.nsteps; ++i) {
-        ok = warp_wait_all(bar(B_DQFULL), (gs + i) & 1, wc);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t v0[32], v1[32];
-        if (live_rows) {
-          tmem_ld32(src, v0);
-          tmem_ld32(src + 32, v1);
-          tmem_wait_ld();
-        }
-        tc_fence_before();
-        mbar_arrive(bar(B_DQEMPTY));
-        if (!live_rows) continue;
-        const int h = step_head(U, i), q0 = step_qblk(U, i) * C::BM;
-        const int nvalid = min(C::BM, p.Nq - q0);
-        float *acc = p.dq_acc + (((size_t)(U.b * p.Hq + h)) * p.Nq + q0 + ch0 * 32) * C::D + t;
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (ch0 * 32 + c < nvalid) atomicAdd(acc + (size_t)c * C::D, __uint_as_float(v0[c]));
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (ch0 * 32 + 32 + c < nvalid) atomicAdd(acc + (size_t)(32 + c) * C::D, __uint_as_float(v1[c]));
+    // Units of the sequence by turn, fetched from the queue by whichever
+    // cursor reaches a turn first (the mask cursor runs at most two steps
+    // ahead of the readout cursor, so eight entries are plenty).
+    int ucache[8];
+    int fetched = 0;
+    auto unit_of = [&](int k, int &u) {
+      while (fetched <= k) {
+        if (!warp_wait_all(bar(B_UFULL + (fetched & 3)), (fetched >> 2) & 1, wc)) return false;
+        ucache[fetched & 7] = s_queue[fetched & 3];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_UEMPTY + (fetched & 3)));
+        ++fetched;
       }
-      gs += U.nsteps;
+      u = ucache[k & 7];
+      return true;
+    };
+    // A cursor over the steps of the sequence: turn k, its unit U, step i of
+    // the unit and g, the running step count (the elementwise stage's gs + i).
+    struct Cursor {
+      int k, i, g;
+      bool end;
+      Unit U;
+    };
+    auto advance = [&](Cursor &c) {
+      if (c.end) return true;
+      if (c.k >= 0 && c.i + 1 < c.U.nsteps) {
+        ++c.i;
+        ++c.g;
+        return true;
+      }
+      for (;;) {
+        int u;
+        if (!unit_of(c.k + 1, u)) return false;
+        ++c.k;
+        if (u < 0) {
+          c.end = true;
+          return true;
+        }
+        c.U = decode(u);
+        if (c.U.nsteps > 0) {
+          c.i = 0;
+          ++c.g;
+          return true;
+        }
+      }
+    };
+    // Dropout keep bits of step c.g: thread tt evaluates the Philox counters
+    // of key rows 4 kq .. 4 kq + 3 (counter word 0 = key / 4, word j of the
+    // result = key row 4 kq + j) for query columns 16 qg .. 16 qg + 15 of the
+    // step, the counters the forward used, and stores 16 bits per key row.
+    auto gen_mask = [&](const Cursor &c) {
+      const int buf = c.g & 1;
+      if (!warp_wait_all(bar(B_MEMPTY + buf), ((c.g >> 1) & 1) ^ 1, wc)) return false;
+      const int tt = (warp - C::READOUT_WARP0) * 32 + lane;
+      const int kq = tt >> 3, qg = tt & 7;
+      const uint32_t kc = (uint32_t)((c.U.kv0 >> 2) + kq);
+      const uint32_t q = (uint32_t)(step_qblk(c.U, c.i) * C::BM + 16 * qg);
+      const uint32_t bhq = (uint32_t)(c.U.b * p.Hq + step_head(c.U, c.i));
+      uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll 4
+      for (int e = 0; e < 16; ++e) {
+        const uint4 R = philox4x32_10(kc, q + e, bhq, p.drop_off, p.seed_lo, p.seed_hi);
+        m0 |= (R.x >= p.drop_thr ? 1u : 0u) << e;
+        m1 |= (R.y >= p.drop_thr ? 1u : 0u) << e;
+        m2 |= (R.z >= p.drop_thr ? 1u : 0u) << e;
+        m3 |= (R.w >= p.drop_thr ? 1u : 0u) << e;
+      }
+      // row r of the buffer: BM bits, 16-bit piece qg = columns 16 qg .. 16 qg + 15
+      uint16_t *mb = reinterpret_cast<uint16_t *>(smem + C::OFF_MASK + buf * C::MASK_BUF) +
+                     (4 * kq) * (C::BM / 16) + qg;
+      mb[0] = (uint16_t)m0;
+      mb[C::BM / 16] = (uint16_t)m1;
+      mb[2 * (C::BM / 16)] = (uint16_t)m2;
+      mb[3 * (C::BM / 16)] = (uint16_t)m3;
+      mbar_arrive(bar(B_MFULL + buf));
+      return true;
+    };
+    // dQ^T of step i of unit U (running step count gi): into registers, TMEM
+    // released, then float32 reductions into the accumulator
+    auto readout = [&](const Unit &U, int i, int gi) {
+      if (!warp_wait_all(bar(B_DQFULL), gi & 1, wc)) return false;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      if (live_rows) {
+        tmem_ld32(src, v0);
+        tmem_ld32(src + 32, v1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_DQEMPTY));
+      if (!live_rows) return true;
+      const int h = step_head(U, i), q0 = step_qblk(U, i) * C::BM;
+      const int nvalid = min(C::BM, p.Nq - q0);
+      float *acc = p.dq_acc + (((size_t)(U.b * p.Hq + h)) * p.Nq + q0 + ch0 * 32) * C::D + t;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (ch0 * 32 + c < nvalid) atomicAdd(acc + (size_t)c * C::D, __uint_as_float(v0[c]));
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (ch0 * 32 + 32 + c < nvalid) atomicAdd(acc + (size_t)(32 + c) * C::D, __uint_as_float(v1[c]));
+      return true;
+    };
+    if constexpr (!DROP) {
+      int gs = 0;
+      for (int k = 0; ok; ++k) {
+        ok = warp_wait_all(bar(B_UFULL + (k & 3)), (k >> 2) & 1, wc);
+        if (!ok) break;
+        const int u = s_queue[k & 3];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_UEMPTY + (k & 3)));
+        if (u < 0) break;
+        const Unit U = decode(u);
+        for (int i = 0; i < U.nsteps && ok; ++i) ok = readout(U, i, gs + i);
+        gs += U.nsteps;
+      }
+    } else {
+      Cursor cd{-1, 0, -1, false, Unit{}};   // dQ readout
+      Cursor cm{-1, 0, -1, false, Unit{}};   // dropout mask, two steps ahead
+      for (int pre = 0; pre < 2 && ok; ++pre) {
+        ok = advance(cm);
+        if (ok && !cm.end) ok = gen_mask(cm);
+      }
+      while (ok) {
+        ok = advance(cd);
+        if (!ok || cd.end) break;
+        ok = readout(cd.U, cd.i, cd.g);
+        if (ok) ok = advance(cm);
+        if (ok && !cm.end) ok = gen_mask(cm);
+      }
     }
   }
 
@@ -1576,7 +1690,7 @@ int run_dkdv(const AttnArgs &a) {
   p.drop_off = (uint32_t)a.drop_offset;
   p.drop_scale = a.drop_scale;
   if constexpr (WIDE) {
-    auto kern = a.drop_thr != 0 ? bwd_wide_kernel<C, true> : bwd_wide_kernel<C, false>;
+    auto kern = bwd_wide_kernel<C, C::MASKGEN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
       return 5;
@@ -1623,8 +1737,14 @@ int launch_bwd_prep_bf16(const AttnArgs &a) {
 // 8-11% slower than bwd_wide_kernel at d = 64 and 128.)
 int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {
-    case 64: return run_dkdv<BwdWideCfg<64, 4, true>, true>(a);
-    case 128: return run_dkdv<BwdWideCfg<128, 2, false>, true>(a);
+    // dropout: the mask-generating instances (at d = 128 with a one-slot
+    // Q/dO ring, which leaves room for the mask buffers)
+    case 64:
+      return a.drop_thr ? run_dkdv<BwdWideCfg<64, 4, true, true>, true>(a)
+                        : run_dkdv<BwdWideCfg<64, 4, true>, true>(a);
+    case 128:
+      return a.drop_thr ? run_dkdv<BwdWideCfg<128, 1, false, true>, true>(a)
+                        : run_dkdv<BwdWideCfg<128, 2, false>, true>(a);
     case 256: {
       int st = run_dkdv<BwdCfg<256, kDV, 64, 2, 2>, false>(a);
       return st ? st : run_dkdv<BwdCfg<256, kDKDQ, 64, 1, 1>, false>(a);
