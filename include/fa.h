@@ -120,8 +120,7 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *
  *
  * Same tensors, layouts, size rules and errors as fa_fwd / fa_bwd, plus:
  * 0 <= p_drop < 1 (else FA_ERR_INVALID_ARG); p_drop = 0 computes exactly
- * fa_fwd / fa_bwd.  fa_bwd_dropout with p_drop > 0 supports d = 64 and 128
- * (FA_ERR_UNSUPPORTED for d = 256).
+ * fa_fwd / fa_bwd.  Both support d = 64, 128 and 256.
  */
 int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
