@@ -43,7 +43,11 @@
 // Dropout (DROP instances): the stored P keeps only the elements whose
 // Philox4x32-10 word is >= floor(p 2^32) (one counter per four key columns of
 // a row); the row sum uses the undropped P and the epilogue scales O by
-// 1 / (1 - p).
+// 1 / (1 - p).  At d = 64 and 128 the dropout instances hold one Q tile per
+// CTA and warps 4-7 evaluate the counters for the key blocks ahead (FwdCfg
+// MW); measured on B200 against the two-tile kernel whose softmax thread
+// evaluates them (causal B4 H16 N4096 d128, p = 0.1): 0.80 -> 0.73 ms.  At
+// d = 256 the softmax thread still evaluates them.
 //
 // E4M3 instances (C::F8): Q, K, V are one-byte OCP E4M3 codes with one
 // dequantisation factor each.  S = Q K^T runs as tcgen05 kind::f8f6f4 (K = 32
@@ -86,9 +90,15 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // P goes to shared memory, which frees S's TMEM columns as soon as the
 // softmax has read them, so S(j+1) is issued while the softmax of block j
 // still runs.
-template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2>
+// MW (dropout instances with one Q tile per CTA): warps 4-7, which have no
+// tile of their own, evaluate the Philox words of the dropout mask for the
+// key blocks ahead and leave one bit per (query row, key) in a double-
+// buffered array in shared memory, so the softmax thread tests bits instead
+// of evaluating a Philox call per four keys.
+template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2, bool MW_ = false>
 struct FwdCfg {
   static constexpr int D = D_, NT = NT_, BN = BN_, STAGES = STAGES_, ES = ES_;
+  static constexpr bool MW = MW_;
   static constexpr bool F8 = ES == 1;
   static constexpr int DCH = D * ES / 128;                // 128-byte column chunks
   static constexpr int CH_ELEMS = 128 / ES;               // elements per chunk (TMA box width)
@@ -112,11 +122,13 @@ struct FwdCfg {
   static constexpr int P_CHUNK = BM * 128;
   static constexpr int P_TILE = P_CHUNK * (P_ROWB / 128);
   static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;
-  static constexpr int OFF_BAR = OFF_P + NT * P_TILE;
+  static constexpr int MASK_BUF = BM * BN / 8;            // [2][BM rows][BN bits]
+  static constexpr int OFF_MASK = OFF_P + NT * P_TILE;
+  static constexpr int OFF_BAR = OFF_MASK + (MW ? 2 * MASK_BUF : 0);
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NT],
   // p_full[NT], o_full[NT], drain, q_empty, o_empty[NT], s_empty[NT] (S read
-  // out of TMEM), p_empty[NT] (P V done with P)
-  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NT + 1 + 1 + NT + 2 * NT;
+  // out of TMEM), p_empty[NT] (P V done with P), mask_full[2], mask_empty[2]
+  static constexpr int NBAR = 1 + 4 * STAGES + 3 * NT + 1 + 1 + NT + 2 * NT + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem base slot, abort flag
   static constexpr int SMEM = OFF_MISC + 16 + 1024;       // + alignment slack
   // TMEM columns
@@ -129,6 +141,7 @@ struct FwdCfg {
   static_assert(BN == 128, "softmax path assumes 128 columns per block");
   static_assert(ES == 1 || ES == 2, "bf16 or e4m3 operands");
   static_assert(D * ES % 128 == 0, "whole 128-byte rows per chunk");
+  static_assert(!MW || (NT == 1 && ES == 2 && BN == 128), "mask warps: one bf16 tile per CTA");
 };
 
 struct FwdParams {
@@ -166,6 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_DRAIN = B_OFULL + C::NT;
   const int B_QEMPTY = B_DRAIN + 1, B_OEMPTY = B_DRAIN + 2;
   const int B_SEMPTY = B_OEMPTY + C::NT, B_PEMPTY = B_SEMPTY + C::NT;
+  const int B_MFULL = B_PEMPTY + C::NT, B_MEMPTY = B_MFULL + 2;
+  static_assert(!C::MW || DROP, "mask warps only in dropout instances");
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
 
@@ -220,6 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_PEMPTY + t), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(B_MFULL + x), BM);    // the mask threads wrote their rows
+      mbar_init(bar(B_MEMPTY + x), BM);   // the softmax threads read theirs
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -459,6 +478,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(B_SEMPTY + t));
         float *s = reinterpret_cast<float *>(sr);
         const int col_lo = (U.j0 + j) * C::BN;
+        // dropout with mask warps: bit 32 c + b of this row's 128 = key
+        // col_lo + 32 c + b kept
+        uint32_t mbits[4] = {0u, 0u, 0u, 0u};
+        if constexpr (C::MW) {
+          const int gj = g + j;
+          ok = warp_wait_all(bar(B_MFULL + (gj & 1)), (gj >> 1) & 1, wc);
+          if (!ok) break;
+          const uint4 mb = *reinterpret_cast<const uint4 *>(smem + C::OFF_MASK + (gj & 1) * C::MASK_BUF +
+                                                            r * (C::BN / 8));
+          mbits[0] = mb.x; mbits[1] = mb.y; mbits[2] = mb.z; mbits[3] = mb.w;
+          mbar_arrive(bar(B_MEMPTY + (gj & 1)));
+        }
         const bool need_mask =
             (col_lo + C::BN > p.Nk) || (p.causal && col_lo + C::BN - 1 > row_lo + p.causal_off);
         if (need_mask) {
@@ -509,7 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p0 = fast_exp2(x0);
             const float p1 = fast_exp2(x1);
             rs[e & 3] += p0 + p1;
-            if (DROP) {
+            if (DROP && C::MW) {
+              const uint32_t mw = mbits[c];
+              pk[e] = pack_bf16x2(((mw >> (2 * e)) & 1u) ? p0 : 0.f, ((mw >> (2 * e + 1)) & 1u) ? p1 : 0.f);
+            } else if (DROP) {
               if ((e & 1) == 0)
                 rnd = philox4x32_10((uint32_t)(col_lo + c * 32 + 2 * e) >> 2, (uint32_t)row,
                                     (uint32_t)bh, p.drop_off, p.seed_lo, p.seed_hi);
@@ -620,6 +654,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       g += U.nkb;
       ++uq;
     }
+  } else if (C::MW && warp < 8) {
+    // ------------------------------------------------------------ mask
+    // Thread r evaluates the dropout mask of query row r of the tile for the
+    // key blocks in order, up to two blocks ahead of the softmax: counter
+    // (key / 4, query row, b*Hq + h, offset), word key % 4 - the words the
+    // backward regenerates - into bits 4 k .. 4 k + 3 of the row's 128.
+    const int r = threadIdx.x - 4 * 32;
+    bool ok = true;
+    int g = 0;
+    for (int k = 0; ok && k * (int)gridDim.x < total_units; ++k) {
+      const int u = k * (int)gridDim.x +
+                    ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+      if (u >= total_units) continue;
+      const Unit U = decode(u);
+      const uint32_t row = (uint32_t)(U.q_start + r);
+      for (int j = 0; j < U.nkb && ok; ++j) {
+        const int gj = g + j;
+        ok = warp_wait_all(bar(B_MEMPTY + (gj & 1)), ((gj >> 1) & 1) ^ 1, wc);
+        if (!ok) break;
+        const uint32_t c0 = (uint32_t)((U.j0 + j) * C::BN) >> 2;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          // four calls in flight per thread (measured on B200 against 1, 2
+          // and 8: causal B4 H16 N4096 d128, p = 0.1, forward 0.92 / 0.74 /
+          // 0.73 / 1.05 ms for 1 / 2 / 4 / 8)
+#pragma unroll 4
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint4 R = philox4x32_10(c0 + 8 * q4 + kk, row, (uint32_t)U.bh, p.drop_off, p.seed_lo,
+                                          p.seed_hi);
+            const uint32_t nib = (R.x >= p.drop_thr ? 1u : 0u) | (R.y >= p.drop_thr ? 2u : 0u) |
+                                 (R.z >= p.drop_thr ? 4u : 0u) | (R.w >= p.drop_thr ? 8u : 0u);
+            w[q4] |= nib << (4 * kk);
+          }
+        }
+        st_shared_v4(sbase + C::OFF_MASK + (gj & 1) * C::MASK_BUF + r * (C::BN / 8), w[0], w[1], w[2], w[3]);
+        mbar_arrive(bar(B_MFULL + (gj & 1)));
+      }
+      g += U.nkb;
+    }
   }
 
   tc_fence_before();
@@ -676,8 +750,11 @@ int run_fwd(const AttnArgs &a) {
   p.o_scale = a.drop_thr != 0 ? a.drop_scale : (C::F8 ? a.descale_v : 1.f);
   p.err = a.err;
   if (a.drop_thr != 0 && a.splits > 1) return 2;   // dropout only in the plain forward
-  auto kern = fwd_kernel<C, false>;
-  if constexpr (!C::F8)
+  if (a.drop_thr != 0 && !C::MW && C::D != 256) return 2;   // d = 64, 128: the mask-warp instances
+  // dropout: the mask-warp instances (d = 64, 128) or, at d = 256, the
+  // instance whose softmax thread evaluates the mask itself
+  auto kern = fwd_kernel<C, C::MW>;
+  if constexpr (!C::F8 && !C::MW && C::D == 256)
     if (a.drop_thr != 0) kern = fwd_kernel<C, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
@@ -804,8 +881,14 @@ int launch_fwd_e4m3_sm100(const AttnArgs &a) {
 
 int launch_fwd_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {
-    case 64: return run_fwd<FwdCfg<64, 2, 128, 3, 2>>(a);
-    case 128: return run_fwd<FwdCfg<128, 2, 128, 1, 2>>(a);
+    // dropout (not in split mode) at d = 64, 128: one Q tile per CTA, with
+    // warps 4-7 evaluating the mask
+    case 64:
+      return a.drop_thr && a.splits == 1 ? run_fwd<FwdCfg<64, 1, 128, 4, 2, true>>(a)
+                                         : run_fwd<FwdCfg<64, 2, 128, 3, 2>>(a);
+    case 128:
+      return a.drop_thr && a.splits == 1 ? run_fwd<FwdCfg<128, 1, 128, 2, 2, true>>(a)
+                                         : run_fwd<FwdCfg<128, 2, 128, 1, 2>>(a);
     case 256: return run_fwd<FwdCfg<256, 1, 128, 1, 2>>(a);
     default: return 2;
   }
