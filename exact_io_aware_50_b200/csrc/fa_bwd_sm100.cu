@@ -108,8 +108,9 @@ struct BwdCfg {
   static constexpr int OFF_DD = OFF_L2 + QS * ROWVEC;
   static constexpr int OFF_BAR = OFF_DD + QS * ROWVEC;
   // kv_full, kc_full, q_full[QS], q_empty[QS], s_full[2], p_full[2],
-  // dq_full[2], dq_empty[2], final, drain, do_full[QS], do_empty[QS]
-  static constexpr int NBAR = 2 + 2 * QS + 8 + 2 + 2 * QS;
+  // dq_full[2], dq_empty[2], final, drain, do_full[QS], do_empty[QS],
+  // acc_empty
+  static constexpr int NBAR = 2 + 2 * QS + 8 + 2 + 2 * QS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
   // so no alignment slack is reserved.
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_KV = 0, B_KC = 1, B_QFULL = 2, B_QEMPTY = 2 + C::QS, B_SFULL = 2 + 2 * C::QS,
             B_PFULL = B_SFULL + 2, B_DQFULL = B_PFULL + 2, B_DQEMPTY = B_DQFULL + 2,
             B_FINAL = B_DQEMPTY + 2, B_DRAIN = B_FINAL + 1, B_DOFULL = B_DRAIN + 1,
-            B_DOEMPTY = B_DOFULL + C::QS;
+            B_DOEMPTY = B_DOFULL + C::QS, B_ACCEMPTY = B_DOEMPTY + C::QS;
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
   const float *s_l2 = (const float *)(smem + C::OFF_L2);
@@ -230,22 +231,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
 
-  // Work unit: head by head (batch, key/value head), and inside a head the
-  // key blocks with the most query blocks first (causal).  A wave then reads
-  // the Q, dO and dQ-accumulator tiles of a few heads only, which stay in L2.
-  const int unit = blockIdx.x;
-  const int jblk = unit % p.nkb;
-  const int bhkv = unit / p.nkb;
-  const int b = bhkv / p.Hkv, hkv = bhkv % p.Hkv;
+  // Work units: (batch, key/value head, key block), head by head, inside a
+  // head the key blocks with the most query blocks first (causal), so a wave
+  // reads the Q, dO and dQ-accumulator tiles of a few heads, which stay in
+  // L2.  Persistent CTAs (one per SM when there are more units): round k
+  // gives CTA c unit k G + c (k even) or k G + G - 1 - c (k odd), G =
+  // gridDim.x, so each CTA keeps its TMEM and barriers and the next unit's
+  // first Q/dO tiles and K/V loads overlap the current unit's last steps and
+  // epilogue.  Barrier phases follow the count of units with work (uc) and
+  // of steps (gs) this CTA has processed.
+  const int total_units = p.nkb * p.BHkv;
+  const int G = (int)gridDim.x;
   const int g = p.Hq / p.Hkv;
-  const int kv0 = jblk * C::BN;
-  const int i0 = p.causal ? kv0 / C::BM : 0;  // first query block that sees this key block
-  const int nq_eff = p.nqb - i0;
-  const int nsteps = nq_eff > 0 ? g * nq_eff : 0;
-  auto step_head = [&](int s) { return hkv * g + s / nq_eff; };
-  auto step_qblk = [&](int s) { return i0 + s % nq_eff; };
-  auto set_of = [&](int s) { return C::NSETS == 2 ? (s & 1) : 0; };
-  auto set_phase = [&](int s) { return (uint32_t)((C::NSETS == 2 ? (s >> 1) : s) & 1); };
+  struct Unit {
+    int bhkv, b, hkv, kv0, i0, nq_eff, nsteps;
+  };
+  auto decode = [&](int u) {
+    Unit U;
+    const int jblk = u % p.nkb;
+    U.bhkv = u / p.nkb;
+    U.b = U.bhkv / p.Hkv;
+    U.hkv = U.bhkv % p.Hkv;
+    U.kv0 = jblk * C::BN;
+    U.i0 = p.causal ? U.kv0 / C::BM : 0;   // first query block that sees this key block
+    U.nq_eff = p.nqb - U.i0;
+    U.nsteps = U.nq_eff > 0 ? g * U.nq_eff : 0;
+    return U;
+  };
+  auto unit_at = [&](int k) {
+    return k * G + ((k & 1) ? G - 1 - (int)blockIdx.x : (int)blockIdx.x);
+  };
+  auto step_head = [&](const Unit &U, int s) { return U.hkv * g + s / U.nq_eff; };
+  auto step_qblk = [&](const Unit &U, int s) { return U.i0 + s % U.nq_eff; };
+  // score set and its barrier phase of the gi-th step of this CTA
+  auto set_of = [&](int gi) { return C::NSETS == 2 ? (gi & 1) : 0; };
+  auto set_phase = [&](int gi) { return (uint32_t)((C::NSETS == 2 ? (gi >> 1) : gi) & 1); };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_KV), 1);
@@ -264,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(B_FINAL), 1);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_ACCEMPTY), 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -289,13 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int last_q[C::QS], last_do[C::QS];
       for (int s = 0; s < C::QS; ++s) last_q[s] = last_do[s] = -1;
+      int kv_phase = -1;
       bool ok = true;
-      mbar_arrive_expect_tx(bar(B_KV), (C::HAS_DP ? 2 : 1) * C::KV_TILE);
-      for (int c = 0; c < C::DCH; ++c) {
-        tma_load_3d(sbase + C::OFF_K + c * C::KV_CHUNK, &tmK, bar(B_KV), c * 64, kv0, bhkv);
-        if (C::HAS_DP)
-          tma_load_3d(sbase + C::OFF_V + c * C::KV_CHUNK, &tmV, bar(B_KV), c * 64, kv0, bhkv);
-      }
+      int uc = 0, gs = 0;
       // Q_i and dO_i fill separate slots.  dK/dQ pass: Q_i carries the row
       // vectors L2_i, D_i (read by the elementwise stage, Q_i last read by
       // dK(i)) and dO_i is read only by dP^T(i), so dO_{i+1} can arrive as soon
@@ -304,50 +321,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dV(i)), so Q_{i+2} can arrive while step i's elementwise work runs.
       constexpr uint32_t ROWS_Q = C::HAS_DP ? 2 * C::ROWVEC : 0;
       constexpr uint32_t ROWS_DO = C::HAS_DP ? 0 : 2 * C::ROWVEC;
-      auto load_rows = [&](int i, int st, uint32_t fb) {
-        const int bh = b * p.Hq + step_head(i);
-        const size_t vrow = (size_t)bh * p.npad + (size_t)step_qblk(i) * C::BM;
+      auto load_rows = [&](const Unit &U, int i, int st, uint32_t fb) {
+        const int bh = U.b * p.Hq + step_head(U, i);
+        const size_t vrow = (size_t)bh * p.npad + (size_t)step_qblk(U, i) * C::BM;
         bulk_load(sbase + C::OFF_L2 + st * C::ROWVEC, p.l2 + vrow, C::ROWVEC, fb);
         bulk_load(sbase + C::OFF_DD + st * C::ROWVEC, p.dsum + vrow, C::ROWVEC, fb);
       };
-      auto load_q = [&](int i, int st, uint32_t ph) {
+      auto load_q = [&](const Unit &U, int i, int st, uint32_t ph) {
         if (!bounded_wait(bar(B_QEMPTY + st), ph ^ 1, wc)) return false;
-        const int bh = b * p.Hq + step_head(i), qb = step_qblk(i);
+        const int bh = U.b * p.Hq + step_head(U, i), qb = step_qblk(U, i);
         const uint32_t fb = bar(B_QFULL + st);
         mbar_arrive_expect_tx(fb, C::Q_TILE + ROWS_Q);
         for (int c = 0; c < C::DCH; ++c)
           tma_load_3d(sbase + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, fb, c * 64,
                       qb * C::BM, bh);
-        if (ROWS_Q) load_rows(i, st, fb);
+        if (ROWS_Q) load_rows(U, i, st, fb);
         last_q[st] = ph;
         return true;
       };
-      auto load_do = [&](int i, int st, uint32_t ph) {
+      auto load_do = [&](const Unit &U, int i, int st, uint32_t ph) {
         if (!bounded_wait(bar(B_DOEMPTY + st), ph ^ 1, wc)) return false;
-        const int bh = b * p.Hq + step_head(i), qb = step_qblk(i);
+        const int bh = U.b * p.Hq + step_head(U, i), qb = step_qblk(U, i);
         const uint32_t fb = bar(B_DOFULL + st);
         mbar_arrive_expect_tx(fb, C::Q_TILE + ROWS_DO);
         for (int c = 0; c < C::DCH; ++c)
           tma_load_3d(sbase + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmDO, fb, c * 64,
                       qb * C::BM, bh);
-        if (ROWS_DO) load_rows(i, st, fb);
+        if (ROWS_DO) load_rows(U, i, st, fb);
         last_do[st] = ph;
         return true;
       };
-      for (int i = 0; i < nsteps && ok; ++i) {
-        const int st = i % C::QS;
-        const uint32_t ph = (i / C::QS) & 1;
-        // the slot freed first goes first: dO in the dK/dQ pass, Q in the dV pass
-        if (C::HAS_DP) {
-          ok = load_do(i, st, ph);
-          if (ok) ok = load_q(i, st, ph);
-        } else {
-          ok = load_q(i, st, ph);
-          if (ok) ok = load_do(i, st, ph);
+      // step i of unit U: the slot freed first goes first (dO in the dK/dQ
+      // pass, Q in the dV pass)
+      auto load_step = [&](const Unit &U, int i) {
+        const int gi = gs + i;
+        const int st = gi % C::QS;
+        const uint32_t ph = (gi / C::QS) & 1;
+        if (C::HAS_DP) return load_do(U, i, st, ph) && load_q(U, i, st, ph);
+        return load_q(U, i, st, ph) && load_do(U, i, st, ph);
+      };
+      for (int k = 0; ok && k * G < total_units; ++k) {
+        const int u = unit_at(k);
+        if (u >= total_units) continue;
+        const Unit U = decode(u);
+        if (U.nsteps == 0) continue;
+        // the first ring slots of this unit, then K (and V) once the previous
+        // unit's MMAs, the last readers of K and V, are done, then the rest
+        const int pre = min(C::QS, U.nsteps);
+        for (int i = 0; i < pre && ok; ++i) ok = load_step(U, i);
+        if (ok && uc > 0) ok = bounded_wait(bar(B_FINAL), (uc - 1) & 1, wc);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(B_KV), (C::HAS_DP ? 2 : 1) * C::KV_TILE);
+        for (int c = 0; c < C::DCH; ++c) {
+          tma_load_3d(sbase + C::OFF_K + c * C::KV_CHUNK, &tmK, bar(B_KV), c * 64, U.kv0, U.bhkv);
+          if (C::HAS_DP)
+            tma_load_3d(sbase + C::OFF_V + c * C::KV_CHUNK, &tmV, bar(B_KV), c * 64, U.kv0, U.bhkv);
         }
+        kv_phase = uc & 1;
+        for (int i = pre; i < U.nsteps && ok; ++i) ok = load_step(U, i);
+        // the next unit's K (and V) go to L2 now, so their load after this
+        // unit's last MMA does not wait on DRAM
+        const int un = unit_at(k + 1);
+        if (ok && (k + 1) * G < total_units && un < total_units) {
+          const Unit N = decode(un);
+          for (int c = 0; c < C::DCH; ++c) {
+            tma_prefetch_l2_3d(&tmK, c * 64, N.kv0, N.bhkv);
+            if (C::HAS_DP) tma_prefetch_l2_3d(&tmV, c * 64, N.kv0, N.bhkv);
+          }
+        }
+        gs += U.nsteps;
+        ++uc;
       }
       if (!ok) {
-        (void)drain_wait(bar(B_KV), 0, p.err, kWaitLimitNs);
+        if (kv_phase >= 0) (void)drain_wait(bar(B_KV), kv_phase, p.err, kWaitLimitNs);
         for (int s = 0; s < C::QS; ++s) {
           if (last_q[s] >= 0) (void)drain_wait(bar(B_QFULL + s), last_q[s], p.err, kWaitLimitNs);
           if (last_do[s] >= 0) (void)drain_wait(bar(B_DOFULL + s), last_do[s], p.err, kWaitLimitNs);
@@ -427,16 +473,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                  IDESC_DQ, kk > 0);
       }
     };
-    // S^T(i) (and dP^T(i) in the dK/dQ pass) into score set x.  The caller
-    // has waited for Q_i; in the dV pass Q_i's slot is released once S^T(i)
-    // is done with it.  dO_i is waited for here and, in the dK/dQ pass, its
-    // slot released once dP^T(i) is done with it.
-    auto issue_scores = [&](int x, int i) {
-      const int st = i % C::QS;
+    // S^T (and dP^T in the dK/dQ pass) of the gi-th step into score set x.
+    // The caller has waited for Q; in the dV pass Q's slot is released once
+    // S^T is done with it.  dO is waited for here and, in the dK/dQ pass, its
+    // slot released once dP^T is done with it.
+    auto issue_scores = [&](int x, int gi) {
+      const int st = gi % C::QS;
       issue_S(x, st);
       if (!C::HAS_DP) mma_commit(bar(B_QEMPTY + st));
       if (C::HAS_DP) {
-        if (!bounded_wait(bar(B_DOFULL + st), (i / C::QS) & 1, wc)) return false;
+        if (!bounded_wait(bar(B_DOFULL + st), (gi / C::QS) & 1, wc)) return false;
         tc_fence_after();
         issue_dP(x, st);
         mma_commit(bar(B_DOEMPTY + st));
@@ -446,263 +492,313 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // The whole role runs in lane 0; the other lanes wait at the end.
     if (lane == 0) {
-    // K - c must be in place before the first MMA reads K
-    bool ok = bounded_wait(bar(B_KC), 0, wc);
-    if (ok && nsteps > 0) {
-      ok = bounded_wait(bar(B_QFULL + 0), 0, wc);
-      if (ok) {
+      bool ok = true;
+      int uc = 0, gs = 0;
+      for (int k = 0; ok && k * G < total_units; ++k) {
+        const int u = unit_at(k);
+        if (u >= total_units) continue;
+        const Unit U = decode(u);
+        const int nsteps = U.nsteps;
+        if (nsteps == 0) continue;
+        // this unit's K - c in place, its first Q loaded
+        ok = bounded_wait(bar(B_KC), uc & 1, wc);
+        if (ok) ok = bounded_wait(bar(B_QFULL + gs % C::QS), (gs / C::QS) & 1, wc);
+        if (!ok) break;
         tc_fence_after();
-        ok = issue_scores(0, 0);
-      }
-    }
-    for (int i = 0; i < nsteps && ok; ++i) {
-      const int x = set_of(i);
-      const int st = i % C::QS;
-      if (C::NSETS == 2 && i + 1 < nsteps) {
-        const int y = x ^ 1;
-        if (C::HAS_DQ && i >= 1) {
-          ok = bounded_wait(bar(B_DQEMPTY + y), set_phase(i - 1), wc);
+        ok = issue_scores(set_of(gs), gs);
+        for (int i = 0; i < nsteps && ok; ++i) {
+          const int gi = gs + i;
+          const int x = set_of(gi);
+          const int st = gi % C::QS;
+          if (C::NSETS == 2 && i + 1 < nsteps) {
+            const int y = x ^ 1;
+            if (C::HAS_DQ && gi >= 1) {
+              ok = bounded_wait(bar(B_DQEMPTY + y), set_phase(gi - 1), wc);
+              if (!ok) break;
+            }
+            const int st1 = (gi + 1) % C::QS;
+            ok = bounded_wait(bar(B_QFULL + st1), ((gi + 1) / C::QS) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            ok = issue_scores(y, gi + 1);
+            if (!ok) break;
+          }
+          ok = bounded_wait(bar(B_PFULL + x), set_phase(gi), wc);
           if (!ok) break;
+          if (C::HAS_DQ && C::NSETS == 1 && gi >= 1) {
+            ok = bounded_wait(bar(B_DQEMPTY + x), set_phase(gi - 1), wc);
+            if (!ok) break;
+          }
+          if (!C::HAS_DP) {
+            // the dV pass reads dO_i in dV(i)
+            ok = bounded_wait(bar(B_DOFULL + st), (gi / C::QS) & 1, wc);
+            if (!ok) break;
+          }
+          // the unit's first dV/dK start the accumulators afresh: the previous
+          // unit's epilogue must have read them out of TMEM
+          if (i == 0 && uc > 0) {
+            ok = bounded_wait(bar(B_ACCEMPTY), (uc - 1) & 1, wc);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          issue_dvdk(x, st, i == 0);
+          // dK/dQ pass: Q_i is done with once dK(i) has read it, and the
+          // elementwise stage finished with L2_i and D_i before p_full; dQ^T(i)
+          // reads K and dS^T only.  dV pass: dO_i and its row vectors likewise.
+          mma_commit(bar(C::HAS_DP ? B_QEMPTY + st : B_DOEMPTY + st));
+          if (C::HAS_DQ) {
+            issue_dq(x);
+            mma_commit(bar(B_DQFULL + x));
+          }
+          if (C::NSETS == 1 && i + 1 < nsteps) {
+            // S^T(i+1) only overwrites P^T/dS^T, which dV/dK(i) (issued
+            // earlier) consume in order; Q_{i+1} arrives while dQ^T(i) runs
+            const int st1 = (gi + 1) % C::QS;
+            ok = bounded_wait(bar(B_QFULL + st1), ((gi + 1) / C::QS) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            ok = issue_scores(x, gi + 1);
+            if (!ok) break;
+          }
         }
-        const int st1 = (i + 1) % C::QS;
-        ok = bounded_wait(bar(B_QFULL + st1), ((i + 1) / C::QS) & 1, wc);
         if (!ok) break;
-        tc_fence_after();
-        ok = issue_scores(y, i + 1);
-        if (!ok) break;
+        // the unit's accumulators are final once its MMAs complete; this
+        // also releases K and V to the producer
+        mma_commit(bar(B_FINAL));
+        gs += nsteps;
+        ++uc;
       }
-      ok = bounded_wait(bar(B_PFULL + x), set_phase(i), wc);
-      if (!ok) break;
-      if (C::HAS_DQ && C::NSETS == 1 && i >= 1) {
-        ok = bounded_wait(bar(B_DQEMPTY + x), set_phase(i - 1), wc);
-        if (!ok) break;
-      }
-      if (!C::HAS_DP) {
-        // the dV pass reads dO_i in dV(i)
-        ok = bounded_wait(bar(B_DOFULL + st), (i / C::QS) & 1, wc);
-        if (!ok) break;
-      }
-      tc_fence_after();
-      issue_dvdk(x, st, i == 0);
-      // dK/dQ pass: Q_i is done with once dK(i) has read it, and the
-      // elementwise stage finished with L2_i and D_i before p_full; dQ^T(i)
-      // reads K and dS^T only.  dV pass: dO_i and its row vectors likewise.
-      mma_commit(bar(C::HAS_DP ? B_QEMPTY + st : B_DOEMPTY + st));
-      if (C::HAS_DQ) {
-        issue_dq(x);
-        mma_commit(bar(B_DQFULL + x));
-      }
-      if (C::NSETS == 1 && i + 1 < nsteps) {
-        // S^T(i+1) only overwrites P^T/dS^T, which dV/dK(i) (issued earlier)
-        // consume in order; Q_{i+1} arrives while dQ^T(i) runs
-        const int st1 = (i + 1) % C::QS;
-        ok = bounded_wait(bar(B_QFULL + st1), ((i + 1) / C::QS) & 1, wc);
-        if (!ok) break;
-        tc_fence_after();
-        ok = issue_scores(x, i + 1);
-        if (!ok) break;
-      }
-    }
-    if (ok) {
-      mma_commit(bar(B_FINAL));
-    } else {
-      {
+      if (!ok) {
         mma_commit(bar(B_DRAIN));
         (void)drain_wait(bar(B_DRAIN), 0, p.err, kWaitLimitNs);
       }
-    }
     }
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------ elementwise stage
     const int wg = warp >> 2;                      // query columns [32 wg, 32 wg + 32)
     const int r = threadIdx.x & 127;               // key row within the block = TMEM lane
-    const int kv = kv0 + r;
-    const bool kv_live = kv < p.Nk;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    // K row r -> K - c in place (same swizzled layout; rows past Nk were
-    // zero-filled and stay zero).  Warpgroup wg takes the 64-column chunks
-    // ch = wg, wg + 2, ...
-    bool ok = warp_wait_all(bar(B_KV), 0, wc);
-    if (ok) {
-      const float *cv = p.cvec + (size_t)bhkv * C::D;
-#pragma unroll 1
-      for (int ch = wg; ch < C::DCH; ch += 2) {
-        uint8_t *row = smem + C::OFF_K + ch * C::KV_CHUNK + r * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int col = ch * 64 + ((u ^ (r & 7)) << 3);
-          const float4 c_lo = *reinterpret_cast<const float4 *>(cv + col);
-          const float4 c_hi = *reinterpret_cast<const float4 *>(cv + col + 4);
-          const float cc[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
-          uint4 v = *reinterpret_cast<const uint4 *>(row + (u << 4));
-          uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
-            const float2 f = __bfloat1622float2(h2);
-            w[e] = kv_live ? pack_bf16x2(f.x - cc[2 * e], f.y - cc[2 * e + 1]) : 0u;
-          }
-          *reinterpret_cast<uint4 *>(row + (u << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_KC));
-    }
-    constexpr int NCB = C::BM / 64;   // 32-column blocks per warpgroup and step
-    for (int i = 0; i < nsteps && ok; ++i) {
-      const int x = set_of(i), st = i % C::QS;
-      // the row vectors L2_i, D_i come with Q_i (dK/dQ pass) or dO_i (dV pass)
-      ok = warp_wait_all(bar((C::HAS_DP ? B_QFULL : B_DOFULL) + st), (i / C::QS) & 1, wc);
-      if (ok) ok = warp_wait_all(bar(B_SFULL + x), set_phase(i), wc);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t set = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE;
-#pragma unroll 1
-      for (int hh = 0; hh < NCB; ++hh) {
-        const int cb = wg * NCB + hh;   // 32-column block of the step
-        const int c0 = cb * 32;
-        uint32_t sv[32], dv[32];
-        tmem_ld32(set + c0, sv);
-        if (C::HAS_DP) tmem_ld32(set + C::TM_DP + c0, dv);
-        tmem_wait_ld();
-        const float4 *l4 = reinterpret_cast<const float4 *>(s_l2 + st * C::BM + c0);
-        const float4 *d4 = reinterpret_cast<const float4 *>(s_dd + st * C::BM + c0);
-        const int q0 = step_qblk(i) * C::BM + c0;
-        // causal: key kv is hidden from query q when kv > q; key rows past
-        // Nk (zero-filled) are masked so they add nothing anywhere.  Query
-        // rows past Nq have L2 = +inf, so their P is 0.
-        const int first_vis = !kv_live ? 32 : (p.causal ? kv - q0 : 0);
-        const bool unmasked = __all_sync(0xffffffffu, first_vis <= 0);
-        // dropout: bit c = query column q0 + c kept for this key row (the same
-        // Philox words the forward used); the dV pass stores P^T * Z, the dK /
-        // dQ pass scales the kept dP^T by 1 / (1 - p)
-        uint32_t keep = 0xffffffffu;
-        if (DROP) {
-          keep = 0u;
-          const uint32_t bhq = (uint32_t)(b * p.Hq + step_head(i));
-#pragma unroll
-          for (int gq = 0; gq < 8; ++gq) keep |= dropout_keep4(kv, q0 + 4 * gq, bhq, p, lane) << (4 * gq);
-        }
-        uint32_t pk[16], dk[16];
-        auto body = [&](auto masked_tag) {
-          constexpr bool MASKED = decltype(masked_tag)::value;
-#pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 lq = l4[e4];
-            const float4 dq4 = C::HAS_DP ? d4[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
-            const float dvv[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
-            float pr[4], ds[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int c = 4 * e4 + u;
-              float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[u]));
-              if (MASKED) pv = (c >= first_vis) ? pv : 0.f;
-              const bool kept = !DROP || ((keep >> c) & 1u);
-              pr[u] = kept ? pv : 0.f;
-              float dpv = __uint_as_float(dv[c]);
-              if (DROP) dpv = kept ? dpv * p.drop_scale : 0.f;
-              ds[u] = C::HAS_DP ? pv * (dpv - dvv[u]) : 0.f;
-            }
-            pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
-            pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
-            dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
-            dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
-          }
-        };
-        if (unmasked) body(std::false_type{});
-        else body(std::true_type{});
-        // bf16 P^T and dS^T go into the 32 S^T columns just read, so columns
-        // another thread group has not read yet are never touched
-        if (C::HAS_DV) tmem_st16(set + c0, pk);
-        if (C::HAS_DK) tmem_st16(set + c0 + 16, dk);
-        if (C::HAS_DQ) {
-          // dS^T row r -> shared memory (B operand of the dQ^T MMA: 64-column
-          // chunks of 128-byte swizzled rows; 16-byte unit u of row r sits
-          // at unit u ^ (r % 8))
-          uint8_t *dsrow = smem + C::OFF_DS + x * C::DS_TILE + (c0 >> 6) * C::DS_CHUNK + r * 128;
-          const int u0 = (c0 & 63) >> 3;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4 *>(dsrow + (((u0 + c) ^ (r & 7)) << 4)) =
-                make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
-        }
-      }
-      if (C::HAS_DQ) fence_proxy_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_PFULL + x));
-      if (C::HAS_DQ && C::NCH == 4) {
-        // Share of the dQ^T readout: chunk 2 + wg (the readout warpgroup takes
-        // chunks 0 and 1), so every column is in registers before dQ^T's TMEM
-        // columns are released, with room to spare.
-        ok = warp_wait_all(bar(B_DQFULL + x), set_phase(i), wc);
-        if (!ok) break;
-        tc_fence_after();
-        const int ch = 2 + wg;
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ + ch * 32, v);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(B_DQEMPTY + x));
-        const int qb0 = step_qblk(i) * C::BM;
-        float *acc = p.dq_acc + (((size_t)(b * p.Hq + step_head(i))) * p.Nq + qb0) * C::D + r;
-        reduce_dq_chunk<C>(v, acc, ch, r, min(C::BM, p.Nq - qb0));
-      }
-    }
-    // ------------------------------------------------------ epilogue
     // warpgroup 0 writes dV, warpgroup 1 writes dK (one key row per thread)
     const bool mine = wg == 0 ? C::HAS_DV : C::HAS_DK;
-    if (ok) ok = warp_wait_all(bar(B_FINAL), 0, wc);
-    if (ok && nsteps > 0 && mine) {
-      tc_fence_after();
-      const size_t rowoff = ((size_t)bhkv * p.Nk + (kv_live ? kv : 0)) * C::D;
-      const uint32_t src = tmem + lane_off + (wg ? C::TM_DK : C::TM_DV);
-      __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + rowoff;
-      const float mul = wg ? p.scale : (DROP ? p.drop_scale : 1.f);
+    constexpr int NCB = C::BM / 64;   // 32-column blocks per warpgroup and step
+    bool ok = true;
+    int uc = 0, gs = 0;
+    for (int k = 0; ok && k * G < total_units; ++k) {
+      const int u = unit_at(k);
+      if (u >= total_units) continue;
+      const Unit U = decode(u);
+      const int kv = U.kv0 + r;
+      const bool kv_live = kv < p.Nk;
+      if (U.nsteps == 0) {
+        // no query row sees this key block: its gradients are zero
+        if (kv_live && mine) {
+          __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + ((size_t)U.bhkv * p.Nk + kv) * C::D;
+          for (int e = 0; e < C::D / 8; ++e) reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0, 0, 0, 0);
+        }
+        continue;
+      }
+      // K row r -> K - c in place (same swizzled layout; rows past Nk were
+      // zero-filled and stay zero).  Warpgroup wg takes the 64-column chunks
+      // ch = wg, wg + 2, ...
+      ok = warp_wait_all(bar(B_KV), uc & 1, wc);
+      if (!ok) break;
+      {
+        const float *cv = p.cvec + (size_t)U.bhkv * C::D;
 #pragma unroll 1
-      for (int c = 0; c < C::D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(src + c * 32, v);
-        tmem_wait_ld();
-        uint32_t pkd[16];
+        for (int ch = wg; ch < C::DCH; ch += 2) {
+          uint8_t *row = smem + C::OFF_K + ch * C::KV_CHUNK + r * 128;
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pkd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-        if (kv_live) {
-          uint4 *o = reinterpret_cast<uint4 *>(dst + c * 32);
+          for (int u8 = 0; u8 < 8; ++u8) {
+            const int col = ch * 64 + ((u8 ^ (r & 7)) << 3);
+            const float4 c_lo = *reinterpret_cast<const float4 *>(cv + col);
+            const float4 c_hi = *reinterpret_cast<const float4 *>(cv + col + 4);
+            const float cc[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
+            uint4 v = *reinterpret_cast<const uint4 *>(row + (u8 << 4));
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+              const float2 f = __bfloat1622float2(h2);
+              w[e] = kv_live ? pack_bf16x2(f.x - cc[2 * e], f.y - cc[2 * e + 1]) : 0u;
+            }
+            *reinterpret_cast<uint4 *>(row + (u8 << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(B_KC));
+      }
+      for (int i = 0; i < U.nsteps && ok; ++i) {
+        const int gi = gs + i;
+        const int x = set_of(gi), st = gi % C::QS;
+        // the row vectors L2_i, D_i come with Q_i (dK/dQ pass) or dO_i (dV pass)
+        ok = warp_wait_all(bar((C::HAS_DP ? B_QFULL : B_DOFULL) + st), (gi / C::QS) & 1, wc);
+        if (ok) ok = warp_wait_all(bar(B_SFULL + x), set_phase(gi), wc);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t set = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE;
+#pragma unroll 1
+        for (int hh = 0; hh < NCB; ++hh) {
+          const int cb = wg * NCB + hh;   // 32-column block of the step
+          const int c0 = cb * 32;
+          uint32_t sv[32], dv[32];
+          tmem_ld32(set + c0, sv);
+          if (C::HAS_DP) tmem_ld32(set + C::TM_DP + c0, dv);
+          tmem_wait_ld();
+          const float4 *l4 = reinterpret_cast<const float4 *>(s_l2 + st * C::BM + c0);
+          const float4 *d4 = reinterpret_cast<const float4 *>(s_dd + st * C::BM + c0);
+          const int q0 = step_qblk(U, i) * C::BM + c0;
+          // causal: key kv is hidden from query q when kv > q; key rows past
+          // Nk (zero-filled) are masked so they add nothing anywhere.  Query
+          // rows past Nq have L2 = +inf, so their P is 0.
+          const int first_vis = !kv_live ? 32 : (p.causal ? kv - q0 : 0);
+          const bool unmasked = __all_sync(0xffffffffu, first_vis <= 0);
+          // dropout: bit c = query column q0 + c kept for this key row (the same
+          // Philox words the forward used); the dV pass stores P^T * Z, the dK /
+          // dQ pass scales the kept dP^T by 1 / (1 - p)
+          uint32_t keep = 0xffffffffu;
+          if (DROP) {
+            keep = 0u;
+            const uint32_t bhq = (uint32_t)(U.b * p.Hq + step_head(U, i));
+#pragma unroll
+            for (int gq = 0; gq < 8; ++gq) keep |= dropout_keep4(kv, q0 + 4 * gq, bhq, p, lane) << (4 * gq);
+          }
+          uint32_t pk[16], dk[16];
+          auto body = [&](auto masked_tag) {
+            constexpr bool MASKED = decltype(masked_tag)::value;
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 lq = l4[e4];
+              const float4 dq4 = C::HAS_DP ? d4[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+              const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
+              const float dvv[4] = {dq4.x, dq4.y, dq4.z, dq4.w};
+              float pr[4], ds[4];
+#pragma unroll
+              for (int u4 = 0; u4 < 4; ++u4) {
+                const int c = 4 * e4 + u4;
+                float pv = fast_exp2(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lv[u4]));
+                if (MASKED) pv = (c >= first_vis) ? pv : 0.f;
+                const bool kept = !DROP || ((keep >> c) & 1u);
+                pr[u4] = kept ? pv : 0.f;
+                float dpv = __uint_as_float(dv[c]);
+                if (DROP) dpv = kept ? dpv * p.drop_scale : 0.f;
+                ds[u4] = C::HAS_DP ? pv * (dpv - dvv[u4]) : 0.f;
+              }
+              pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
+              pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
+              dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+              dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
+            }
+          };
+          if (unmasked) body(std::false_type{});
+          else body(std::true_type{});
+          // bf16 P^T and dS^T go into the 32 S^T columns just read, so columns
+          // another thread group has not read yet are never touched
+          if (C::HAS_DV) tmem_st16(set + c0, pk);
+          if (C::HAS_DK) tmem_st16(set + c0 + 16, dk);
+          if (C::HAS_DQ) {
+            // dS^T row r -> shared memory (B operand of the dQ^T MMA: 64-column
+            // chunks of 128-byte swizzled rows; 16-byte unit u of row r sits
+            // at unit u ^ (r % 8))
+            uint8_t *dsrow = smem + C::OFF_DS + x * C::DS_TILE + (c0 >> 6) * C::DS_CHUNK + r * 128;
+            const int u0 = (c0 & 63) >> 3;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4 *>(dsrow + (((u0 + c) ^ (r & 7)) << 4)) =
+                  make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+          }
+        }
+        if (C::HAS_DQ) fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + x));
+        if (C::HAS_DQ && C::NCH == 4) {
+          // Share of the dQ^T readout: chunk 2 + wg (the readout warpgroup takes
+          // chunks 0 and 1), so every column is in registers before dQ^T's TMEM
+          // columns are released, with room to spare.
+          ok = warp_wait_all(bar(B_DQFULL + x), set_phase(gi), wc);
+          if (!ok) break;
+          tc_fence_after();
+          const int ch = 2 + wg;
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ + ch * 32, v);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(B_DQEMPTY + x));
+          const int qb0 = step_qblk(U, i) * C::BM;
+          float *acc = p.dq_acc + (((size_t)(U.b * p.Hq + step_head(U, i))) * p.Nq + qb0) * C::D + r;
+          reduce_dq_chunk<C>(v, acc, ch, r, min(C::BM, p.Nq - qb0));
         }
       }
-    } else if (ok && nsteps == 0 && kv_live && mine) {
-      // no query row sees this key block: its gradients are zero
-      __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + ((size_t)bhkv * p.Nk + kv) * C::D;
-      for (int e = 0; e < C::D / 8; ++e) reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0, 0, 0, 0);
+      if (!ok) break;
+      // ---------------------------------------------------- epilogue
+      // the accumulators are released once read, before the stores complete
+      ok = warp_wait_all(bar(B_FINAL), uc & 1, wc);
+      if (!ok) break;
+      tc_fence_after();
+      if (!mine) {
+        tc_fence_before();
+        mbar_arrive(bar(B_ACCEMPTY));
+      } else {
+        const size_t rowoff = ((size_t)U.bhkv * p.Nk + (kv_live ? kv : 0)) * C::D;
+        const uint32_t src = tmem + lane_off + (wg ? C::TM_DK : C::TM_DV);
+        __nv_bfloat16 *dst = (wg ? p.dk : p.dv) + rowoff;
+        const float mul = wg ? p.scale : (DROP ? p.drop_scale : 1.f);
+#pragma unroll 1
+        for (int c = 0; c < C::D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(src + c * 32, v);
+          tmem_wait_ld();
+          if (c == C::D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(B_ACCEMPTY));
+          }
+          uint32_t pkd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pkd[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+          if (kv_live) {
+            uint4 *o = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+          }
+        }
+      }
+      gs += U.nsteps;
+      ++uc;
     }
   } else if (warp < kProducerWarp && C::HAS_DQ) {
     // ------------------------------------------------ dQ readout
     const int t = threadIdx.x - 32 * kReadoutWarp0;  // TMEM lane = column d of dQ (per half)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     static_assert(C::NCH == 2 || C::NCH == 4, "dQ^T readout split");
-    for (int i = 0; i < nsteps; ++i) {
-      const int x = set_of(i);
-      if (!warp_wait_all(bar(B_DQFULL + x), set_phase(i), wc)) break;
-      tc_fence_after();
-      const int h = step_head(i), q0 = step_qblk(i) * C::BM;
-      const int nvalid = min(C::BM, p.Nq - q0);
-      float *acc = p.dq_acc + (((size_t)(b * p.Hq + h)) * p.Nq + q0) * C::D + t;
-      const uint32_t src = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ;
-      // chunks 0 and 1 (the elementwise warpgroups take chunks 2 and 3)
-      uint32_t v0[32], v1[32];
-      tmem_ld32(src, v0);
-      tmem_ld32(src + 32, v1);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_DQEMPTY + x));
-      reduce_dq_chunk<C>(v0, acc, 0, t, nvalid);
-      reduce_dq_chunk<C>(v1, acc, 1, t, nvalid);
+    bool ok = true;
+    int gs = 0;
+    for (int k = 0; ok && k * G < total_units; ++k) {
+      const int u = unit_at(k);
+      if (u >= total_units) continue;
+      const Unit U = decode(u);
+      for (int i = 0; i < U.nsteps && ok; ++i) {
+        const int gi = gs + i;
+        const int x = set_of(gi);
+        ok = warp_wait_all(bar(B_DQFULL + x), set_phase(gi), wc);
+        if (!ok) break;
+        tc_fence_after();
+        const int h = step_head(U, i), q0 = step_qblk(U, i) * C::BM;
+        const int nvalid = min(C::BM, p.Nq - q0);
+        float *acc = p.dq_acc + (((size_t)(U.b * p.Hq + h)) * p.Nq + q0) * C::D + t;
+        const uint32_t src = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ;
+        // chunks 0 and 1 (the elementwise warpgroups take chunks 2 and 3)
+        uint32_t v0[32], v1[32];
+        tmem_ld32(src, v0);
+        tmem_ld32(src + 32, v1);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_DQEMPTY + x));
+        reduce_dq_chunk<C>(v0, acc, 0, t, nvalid);
+        reduce_dq_chunk<C>(v1, acc, 1, t, nvalid);
+      }
+      gs += U.nsteps;
     }
   }
 
@@ -1706,7 +1802,19 @@ int run_dkdv(const AttnArgs &a) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
       return 5;
-    kern<<<(unsigned)units, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
+    // Persistent (one CTA per SM) when units are short, where a CTA's set-up
+    // and epilogue weigh most; otherwise one CTA per unit, whose hardware
+    // order balances the causal units' unequal lengths better than the
+    // static snake.  Measured on B200 (dkdv, B*N = 32768, H16): N = 512
+    // causal 1.334 -> 1.248 ms, N = 2048 causal 3.018 -> 2.798 ms, N = 8192
+    // causal 9.61 -> 9.79 ms with the persistent grid.
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 5;
+    const bool persist = (long long)(a.Hq / a.Hkv) * p.nqb <= 32;
+    const long long grid = persist && units > sms ? sms : units;
+    kern<<<(unsigned)grid, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, mdo, p);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }
@@ -1732,7 +1840,9 @@ int launch_bwd_prep_bf16(const AttnArgs &a) {
 
 
 // d = 64 and 128: one pass with 128-row query blocks (bwd_wide_kernel).
-// d = 256: dK and dV alone fill TMEM, so two passes of bwd_kernel.
+// d = 256: dK and dV alone fill TMEM, so two passes of bwd_kernel (each CTA
+// runs a static snake sequence of units, one unit per CTA when the grid has
+// one CTA per unit).
 // (bwd_kernel's single-pass mode, 64-row blocks in two TMEM sets, measured
 // 8-11% slower than bwd_wide_kernel at d = 64 and 128.)
 int launch_bwd_dkdv_bf16_sm100(const AttnArgs &a) {
