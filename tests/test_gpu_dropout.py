@@ -48,7 +48,11 @@ def test_dropout_mask_bits():
 
 CASES = [(1, 2, 1, 300, 64, True, 0.1), (2, 2, 2, 257, 128, False, 0.5),
          (1, 4, 2, 513, 128, True, 0.3), (1, 2, 1, 300, 256, True, 0.2),
-         (2, 2, 2, 200, 256, False, 0.4)]
+         (2, 2, 2, 200, 256, False, 0.4),
+         # more units than SMs: the mask warps and the readout warps' mask
+         # cursors cross unit boundaries, and the d = 256 passes run persistently
+         (24, 4, 2, 400, 128, True, 0.2), (24, 4, 2, 400, 64, True, 0.1),
+         (32, 4, 2, 400, 256, False, 0.3)]
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "x".join(str(v) for v in c))

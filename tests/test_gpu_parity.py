@@ -125,6 +125,23 @@ def test_bf16_backward_small(shape):
     run_full_check(B, Hq, Hkv, Nq, Nk, d, causal, "bf16", seed=51)
 
 
+# More key-block units than the B200's 148 SMs, so the persistent backward
+# kernels walk several units per CTA (barrier phases, K/V reloads and the
+# accumulator hand-over across unit boundaries), with GQA and ragged lengths.
+BF16_BWD_MANY_UNITS = [
+    (32, 4, 2, 400, 400, 256, True),     # d = 256, persistent two passes, 256 units
+    (40, 2, 2, 300, 300, 256, False),    # 240 units
+    (24, 4, 2, 400, 400, 128, True),     # d = 128, 192 units
+    (20, 4, 4, 260, 260, 64, False),     # d = 64, 240 units
+]
+
+
+@pytest.mark.parametrize("shape", BF16_BWD_MANY_UNITS, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_backward_many_units(shape):
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    run_full_check(B, Hq, Hkv, Nq, Nk, d, causal, "bf16", seed=61)
+
+
 def test_bf16_backward_sharp_and_shifted():
     run_full_check(1, 4, 1, 1024, 1024, 128, True, "bf16", seed=61, q_mul=2.0)
     run_full_check(1, 2, 2, 768, 768, 128, True, "bf16", seed=62, k_add=8.0)
