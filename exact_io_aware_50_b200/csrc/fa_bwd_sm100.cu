@@ -1627,7 +1627,11 @@ __global__ void bwd_center_kernel(const __nv_bfloat16 *__restrict__ k, float *__
 // Per padded query row: D = sum_d dO * O and
 // L2 = log2e * L - scale * log2e * (q . c) (rows past Nq: D = 0, L2 = +inf);
 // zero the row of the dQ accumulator.  D / 8 lanes per row, each reading 16
-// bytes of O, dO and Q (so a warp covers 32 * 8 / D rows).
+// bytes of O, dO and Q (so a warp covers 32 * 8 / D rows).  A lane reads Q
+// only where its 8 entries of c are not all zero: c is the key mean rounded
+// to integers, zero for keys centred near 0, and the skipped products are
+// exact zeros, so most calls read no Q at all (measured on B200 at causal B4
+// H16 N4096 d128, centring and preprocess together: 64.5 -> 60.4 us).
 template <int D>
 __global__ void bwd_preprocess_kernel(const __nv_bfloat16 *__restrict__ q,
                                       const __nv_bfloat16 *__restrict__ o,
@@ -1653,9 +1657,11 @@ __global__ void bwd_preprocess_kernel(const __nv_bfloat16 *__restrict__ q,
     const float *cv = cvec + ((size_t)b * (Hq / g) + h / g) * D + l * 8;
     const uint4 ov = *reinterpret_cast<const uint4 *>(o + row * D + l * 8);
     const uint4 dv = *reinterpret_cast<const uint4 *>(dout + row * D + l * 8);
-    const uint4 qv = *reinterpret_cast<const uint4 *>(q + row * D + l * 8);
     const float4 c0 = *reinterpret_cast<const float4 *>(cv);
     const float4 c1 = *reinterpret_cast<const float4 *>(cv + 4);
+    const bool need_q = c0.x != 0.f || c0.y != 0.f || c0.z != 0.f || c0.w != 0.f || c1.x != 0.f ||
+                        c1.y != 0.f || c1.z != 0.f || c1.w != 0.f;
+    const uint4 qv = need_q ? *reinterpret_cast<const uint4 *>(q + row * D + l * 8) : make_uint4(0, 0, 0, 0);
     const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w},
                    qw[4] = {qv.x, qv.y, qv.z, qv.w};
     const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
