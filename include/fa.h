@@ -59,7 +59,9 @@ typedef enum {
 } fa_status;
 
 /*
- * fa_fwd -- BF16 forward.  q, k, v, o: bfloat16; lse: float32.
+ * fa_fwd -- BF16 forward: O and L of the operation above, computed tile by
+ * tile with the online softmax and one final normalisation (blog section 4.1
+ * "v2", CSDN tutorial section 3).  q, k, v, o: bfloat16; lse: float32.
  * d must be 64, 128 or 256.  causal != 0 requires Nq == Nk.
  * Nq, Nk >= 1 (any length; tails are masked).  scale is applied to Q K^T
  * before the softmax (1/sqrt(d) for standard attention).
@@ -164,7 +166,8 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
 
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd and fa_bwd_f32
- * need (float32 throughout): the per-row vector D = rowsum(dO * O) and the
+ * need, i.e. what the recomputing backward (blog section 2.3) keeps besides
+ * the inputs (float32 throughout): the per-row vector D = rowsum(dO * O) and the
  * per-row base-2 log-sum-exp used by the backward, each padded to a multiple
  * of 128 rows per head; one centring vector per head (B*Hq*d); a work
  * counter of the persistent main pass; and a dQ accumulator (B*Hq*Nq*d),
@@ -174,7 +177,10 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
 size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
 
 /*
- * fa_bwd -- BF16 backward.  q, k, v, o, dout: bfloat16 (o and lse as written
+ * fa_bwd -- BF16 backward: dQ, dK, dV of f = sum(O * dO) with P recomputed
+ * from Q, K and L instead of stored (blog section 2.3): dV = P^T dO,
+ * dP = dO V^T, dS = P * (dP - D) with D = rowsum(dO * O), dQ = scale dS K,
+ * dK = scale dS^T Q.  q, k, v, o, dout: bfloat16 (o and lse as written
  * by fa_fwd for the same inputs); dq, dk, dv: bfloat16 outputs; workspace:
  * at least fa_bwd_workspace_size(B, Hq, Nq, d) bytes of device memory,
  * 256-byte aligned, contents ignored on entry and clobbered.
