@@ -106,11 +106,14 @@ struct BwdCfg {
   static constexpr int OFF_DS = OFF_DO + QS * Q_TILE;
   static constexpr int OFF_L2 = OFF_DS + (HAS_DQ ? NSETS * DS_TILE : 0);
   static constexpr int OFF_DD = OFF_L2 + QS * ROWVEC;
-  static constexpr int OFF_BAR = OFF_DD + QS * ROWVEC;
+  // dropout keep bits of a step, [128 key rows][BM query bits], two buffers
+  static constexpr int MASK_BUF = BN * BM / 8;
+  static constexpr int OFF_MASK = OFF_DD + QS * ROWVEC;
+  static constexpr int OFF_BAR = OFF_MASK + 2 * MASK_BUF;
   // kv_full, kc_full, q_full[QS], q_empty[QS], s_full[2], p_full[2],
   // dq_full[2], dq_empty[2], final, drain, do_full[QS], do_empty[QS],
-  // acc_empty
-  static constexpr int NBAR = 2 + 2 * QS + 8 + 2 + 2 * QS + 1;
+  // acc_empty, mask_full[2], mask_empty[2]
+  static constexpr int NBAR = 2 + 2 * QS + 8 + 2 + 2 * QS + 1 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
   // so no alignment slack is reserved.
@@ -159,28 +162,6 @@ struct BwdParams {
   unsigned *err;
 };
 
-// Keep bits of the dropout mask for key row kv (this thread) and the four
-// query columns i0 .. i0 + 3 (bit c for column i0 + c).  The four threads of
-// a lane quad hold four consecutive key rows, which share one Philox counter
-// (kv / 4, i): thread l of the quad evaluates the counter of column i0 + l
-// and the quad exchanges words so that each thread gets word kv % 4 of all
-// four columns.  All 32 lanes must call this together.
-__device__ __forceinline__ uint32_t dropout_keep4(int kv, int i0, uint32_t bhq, const BwdParams &p,
-                                                  int lane) {
-  const int l = lane & 3;
-  const uint4 R = philox4x32_10((uint32_t)kv >> 2, (uint32_t)(i0 + l), bhq, p.drop_off, p.seed_lo,
-                                p.seed_hi);
-  auto word = [&](int idx) { return idx == 0 ? R.x : idx == 1 ? R.y : idx == 2 ? R.z : R.w; };
-  uint32_t bits = (word(l) >= p.drop_thr) ? (1u << l) : 0u;
-#pragma unroll
-  for (int k = 1; k < 4; ++k) {
-    // lane l reads from quad lane s = l + k the word s sent, word (s - k) = l
-    const uint32_t got = __shfl_sync(0xffffffffu, word((l - k) & 3), (lane & ~3) | ((l + k) & 3));
-    bits |= (got >= p.drop_thr) ? (1u << ((l + k) & 3)) : 0u;
-  }
-  return bits;
-}
-
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
                                           uint32_t bar) {
   asm volatile(
@@ -222,7 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_KV = 0, B_KC = 1, B_QFULL = 2, B_QEMPTY = 2 + C::QS, B_SFULL = 2 + 2 * C::QS,
             B_PFULL = B_SFULL + 2, B_DQFULL = B_PFULL + 2, B_DQEMPTY = B_DQFULL + 2,
             B_FINAL = B_DQEMPTY + 2, B_DRAIN = B_FINAL + 1, B_DOFULL = B_DRAIN + 1,
-            B_DOEMPTY = B_DOFULL + C::QS, B_ACCEMPTY = B_DOEMPTY + C::QS;
+            B_DOEMPTY = B_DOFULL + C::QS, B_ACCEMPTY = B_DOEMPTY + C::QS,
+            B_MFULL = B_ACCEMPTY + 1, B_MEMPTY = B_MFULL + 2;
   uint32_t *tmem_slot = (uint32_t *)(smem + C::OFF_MISC);
   volatile int *abort_flag = (volatile int *)(smem + C::OFF_MISC + 4);
   const float *s_l2 = (const float *)(smem + C::OFF_L2);
@@ -285,6 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_FINAL), 1);
     mbar_init(bar(B_DRAIN), 1);
     mbar_init(bar(B_ACCEMPTY), 256);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(B_MFULL + x), 128);    // the mask threads wrote their rows
+      mbar_init(bar(B_MEMPTY + x), 256);   // the elementwise threads read theirs
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -637,6 +623,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t set = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE;
+        // dropout: bit c of word cb = query column 32 cb + c of the step kept for
+        // this key row (the Philox words the forward used, evaluated ahead by
+        // warps 8-11); the dV pass stores P^T * Z, the dK / dQ pass scales the
+        // kept dP^T by 1 / (1 - p)
+        uint32_t keepw[NCB];
+        if (DROP) {
+          ok = warp_wait_all(bar(B_MFULL + (gi & 1)), (gi >> 1) & 1, wc);
+          if (!ok) break;
+          const uint32_t *mrow = reinterpret_cast<const uint32_t *>(
+              smem + C::OFF_MASK + (gi & 1) * C::MASK_BUF + r * (C::BM / 8));
+#pragma unroll
+          for (int hh = 0; hh < NCB; ++hh) keepw[hh] = mrow[wg * NCB + hh];
+          mbar_arrive(bar(B_MEMPTY + (gi & 1)));
+        }
 #pragma unroll 1
         for (int hh = 0; hh < NCB; ++hh) {
           const int cb = wg * NCB + hh;   // 32-column block of the step
@@ -653,16 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // rows past Nq have L2 = +inf, so their P is 0.
           const int first_vis = !kv_live ? 32 : (p.causal ? kv - q0 : 0);
           const bool unmasked = __all_sync(0xffffffffu, first_vis <= 0);
-          // dropout: bit c = query column q0 + c kept for this key row (the same
-          // Philox words the forward used); the dV pass stores P^T * Z, the dK /
-          // dQ pass scales the kept dP^T by 1 / (1 - p)
-          uint32_t keep = 0xffffffffu;
-          if (DROP) {
-            keep = 0u;
-            const uint32_t bhq = (uint32_t)(U.b * p.Hq + step_head(U, i));
-#pragma unroll
-            for (int gq = 0; gq < 8; ++gq) keep |= dropout_keep4(kv, q0 + 4 * gq, bhq, p, lane) << (4 * gq);
-          }
+          const uint32_t keep = DROP ? keepw[hh] : 0xffffffffu;
           uint32_t pk[16], dk[16];
           auto body = [&](auto masked_tag) {
             constexpr bool MASKED = decltype(masked_tag)::value;
@@ -767,12 +758,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       gs += U.nsteps;
       ++uc;
     }
-  } else if (warp < kProducerWarp && C::HAS_DQ) {
-    // ------------------------------------------------ dQ readout
+  } else if (warp < kProducerWarp && (C::HAS_DQ || DROP)) {
+    // ---------------------------------- dQ readout and dropout mask
     const int t = threadIdx.x - 32 * kReadoutWarp0;  // TMEM lane = column d of dQ (per half)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    static_assert(C::NCH == 2 || C::NCH == 4, "dQ^T readout split");
+    static_assert(!C::HAS_DQ || C::NCH == 2 || C::NCH == 4, "dQ^T readout split");
+    static_assert(!DROP || C::BM == 64, "mask threads: 32 key quads x 4 groups of 16 query columns");
     bool ok = true;
+    // Dropout mask, two steps ahead of the elementwise stage: the mask cursor
+    // walks the same unit sequence (step mi of the unit at turn mk; mg counts
+    // the steps, the elementwise stage's gi).  Thread t evaluates the Philox
+    // counters of key rows 4 kq .. 4 kq + 3 (counter word 0 = key / 4, word j
+    // of the result = key row 4 kq + j) and query columns 16 qg .. 16 qg + 15.
+    int mk = -1, mi = 0, mg = -1;
+    bool mend = false;
+    Unit mU{};
+    auto madvance = [&]() {
+      if (mk >= 0 && mi + 1 < mU.nsteps) {
+        ++mi;
+        ++mg;
+        return;
+      }
+      for (;;) {
+        ++mk;
+        if (mk * G >= total_units) {
+          mend = true;
+          return;
+        }
+        const int u = unit_at(mk);
+        if (u >= total_units) continue;
+        mU = decode(u);
+        if (mU.nsteps > 0) {
+          mi = 0;
+          ++mg;
+          return;
+        }
+      }
+    };
+    auto gen_mask = [&]() {
+      const int buf = mg & 1;
+      if (!warp_wait_all(bar(B_MEMPTY + buf), ((mg >> 1) & 1) ^ 1, wc)) return false;
+      const int kq = t >> 2, qg = t & 3;
+      const uint32_t kc = (uint32_t)((mU.kv0 >> 2) + kq);
+      const uint32_t q = (uint32_t)(step_qblk(mU, mi) * C::BM + 16 * qg);
+      const uint32_t bhq = (uint32_t)(mU.b * p.Hq + step_head(mU, mi));
+      uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll 4
+      for (int e = 0; e < 16; ++e) {
+        const uint4 R = philox4x32_10(kc, q + e, bhq, p.drop_off, p.seed_lo, p.seed_hi);
+        m0 |= (R.x >= p.drop_thr ? 1u : 0u) << e;
+        m1 |= (R.y >= p.drop_thr ? 1u : 0u) << e;
+        m2 |= (R.z >= p.drop_thr ? 1u : 0u) << e;
+        m3 |= (R.w >= p.drop_thr ? 1u : 0u) << e;
+      }
+      // row r of the buffer: BM bits, 16-bit piece qg = columns 16 qg .. 16 qg + 15
+      uint16_t *mb = reinterpret_cast<uint16_t *>(smem + C::OFF_MASK + buf * C::MASK_BUF) +
+                     (4 * kq) * (C::BM / 16) + qg;
+      mb[0] = (uint16_t)m0;
+      mb[C::BM / 16] = (uint16_t)m1;
+      mb[2 * (C::BM / 16)] = (uint16_t)m2;
+      mb[3 * (C::BM / 16)] = (uint16_t)m3;
+      mbar_arrive(bar(B_MFULL + buf));
+      return true;
+    };
+    if (DROP) {
+      for (int pre = 0; pre < 2 && ok; ++pre) {
+        madvance();
+        if (!mend) ok = gen_mask();
+      }
+    }
     int gs = 0;
     for (int k = 0; ok && k * G < total_units; ++k) {
       const int u = unit_at(k);
@@ -780,23 +834,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit U = decode(u);
       for (int i = 0; i < U.nsteps && ok; ++i) {
         const int gi = gs + i;
-        const int x = set_of(gi);
-        ok = warp_wait_all(bar(B_DQFULL + x), set_phase(gi), wc);
-        if (!ok) break;
-        tc_fence_after();
-        const int h = step_head(U, i), q0 = step_qblk(U, i) * C::BM;
-        const int nvalid = min(C::BM, p.Nq - q0);
-        float *acc = p.dq_acc + (((size_t)(U.b * p.Hq + h)) * p.Nq + q0) * C::D + t;
-        const uint32_t src = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ;
-        // chunks 0 and 1 (the elementwise warpgroups take chunks 2 and 3)
-        uint32_t v0[32], v1[32];
-        tmem_ld32(src, v0);
-        tmem_ld32(src + 32, v1);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(B_DQEMPTY + x));
-        reduce_dq_chunk<C>(v0, acc, 0, t, nvalid);
-        reduce_dq_chunk<C>(v1, acc, 1, t, nvalid);
+        if (C::HAS_DQ) {
+          const int x = set_of(gi);
+          ok = warp_wait_all(bar(B_DQFULL + x), set_phase(gi), wc);
+          if (!ok) break;
+          tc_fence_after();
+          const int h = step_head(U, i), q0 = step_qblk(U, i) * C::BM;
+          const int nvalid = min(C::BM, p.Nq - q0);
+          float *acc = p.dq_acc + (((size_t)(U.b * p.Hq + h)) * p.Nq + q0) * C::D + t;
+          const uint32_t src = tmem + lane_off + C::TM_SET0 + x * C::SET_STRIDE + C::TM_DQ;
+          // chunks 0 and 1 (the elementwise warpgroups take chunks 2 and 3)
+          uint32_t v0[32], v1[32];
+          tmem_ld32(src, v0);
+          tmem_ld32(src + 32, v1);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(B_DQEMPTY + x));
+          reduce_dq_chunk<C>(v0, acc, 0, t, nvalid);
+          reduce_dq_chunk<C>(v1, acc, 1, t, nvalid);
+        }
+        if (DROP) {
+          madvance();
+          if (!mend) ok = gen_mask();
+        }
       }
       gs += U.nsteps;
     }
