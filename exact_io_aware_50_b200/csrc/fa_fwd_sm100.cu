@@ -43,11 +43,10 @@
 // Dropout (DROP instances): the stored P keeps only the elements whose
 // Philox4x32-10 word is >= floor(p 2^32) (one counter per four key columns of
 // a row); the row sum uses the undropped P and the epilogue scales O by
-// 1 / (1 - p).  At d = 64 and 128 the dropout instances hold one Q tile per
-// CTA and warps 4-7 evaluate the counters for the key blocks ahead (FwdCfg
-// MW); measured on B200 against the two-tile kernel whose softmax thread
-// evaluates them (causal B4 H16 N4096 d128, p = 0.1): 0.80 -> 0.73 ms.  At
-// d = 256 the softmax thread still evaluates them.
+// 1 / (1 - p).  The dropout instances hold one Q tile per CTA and warps
+// 4-7 evaluate the counters for the key blocks ahead (FwdCfg MW); measured
+// on B200 against the two-tile kernel whose softmax thread evaluated them
+// (causal B4 H16 N4096 d128, p = 0.1): 0.80 -> 0.73 ms.
 //
 // E4M3 instances (C::F8): Q, K, V are one-byte OCP E4M3 codes with one
 // dequantisation factor each.  S = Q K^T runs as tcgen05 kind::f8f6f4 (K = 32
@@ -122,15 +121,19 @@ struct FwdCfg {
   static constexpr int P_CHUNK = BM * 128;
   static constexpr int P_TILE = P_CHUNK * (P_ROWB / 128);
   static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;
-  static constexpr int MASK_BUF = BM * BN / 8;            // [2][BM rows][BN bits]
+  static constexpr int MASK_BUF = BM * BN / 8;            // [MASK_NBUF][BM rows][BN bits]
+  // d = 256 has room for one mask buffer only (and no alignment slack: the
+  // dynamic shared window is 1024-byte aligned, checked at run time)
+  static constexpr int MASK_NBUF = D >= 256 ? 1 : 2;
+  static constexpr int SLACK = (MW && D >= 256) ? 0 : 1024;
   static constexpr int OFF_MASK = OFF_P + NT * P_TILE;
-  static constexpr int OFF_BAR = OFF_MASK + (MW ? 2 * MASK_BUF : 0);
+  static constexpr int OFF_BAR = OFF_MASK + (MW ? MASK_NBUF * MASK_BUF : 0);
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NT],
   // p_full[NT], o_full[NT], drain, q_empty, o_empty[NT], s_empty[NT] (S read
   // out of TMEM), p_empty[NT] (P V done with P), mask_full[2], mask_empty[2]
   static constexpr int NBAR = 1 + 4 * STAGES + 3 * NT + 1 + 1 + NT + 2 * NT + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem base slot, abort flag
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;       // + alignment slack
+  static constexpr int SMEM = OFF_MISC + 16 + SLACK;      // + alignment slack
   // TMEM columns
   static constexpr int TM_S = 0;                          // S_t at t*BN
   static constexpr int TM_O = NT * BN;                    // O_t at TM_O + t*D
@@ -167,7 +170,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   static_assert(!(DROP && C::F8), "dropout is built for the bf16 forward only");
-  extern __shared__ uint8_t smem_raw[];
+  static_assert(DROP == C::MW, "dropout instances take their mask from the mask warps");
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (C::SLACK == 0 && (smem_u32(smem_raw) & 1023u)) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrConfig);
+    return;
+  }
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
   uint64_t *bars = (uint64_t *)(smem + C::OFF_BAR);
@@ -483,12 +491,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t mbits[4] = {0u, 0u, 0u, 0u};
         if constexpr (C::MW) {
           const int gj = g + j;
-          ok = warp_wait_all(bar(B_MFULL + (gj & 1)), (gj >> 1) & 1, wc);
+          const int mbuf = gj % C::MASK_NBUF;
+          ok = warp_wait_all(bar(B_MFULL + mbuf), (gj / C::MASK_NBUF) & 1, wc);
           if (!ok) break;
-          const uint4 mb = *reinterpret_cast<const uint4 *>(smem + C::OFF_MASK + (gj & 1) * C::MASK_BUF +
+          const uint4 mb = *reinterpret_cast<const uint4 *>(smem + C::OFF_MASK + mbuf * C::MASK_BUF +
                                                             r * (C::BN / 8));
           mbits[0] = mb.x; mbits[1] = mb.y; mbits[2] = mb.z; mbits[3] = mb.w;
-          mbar_arrive(bar(B_MEMPTY + (gj & 1)));
+          mbar_arrive(bar(B_MEMPTY + mbuf));
         }
         const bool need_mask =
             (col_lo + C::BN > p.Nk) || (p.causal && col_lo + C::BN - 1 > row_lo + p.causal_off);
@@ -532,7 +541,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   #pragma unroll
         for (int c = 0; c < C::BN / 32; ++c) {
           uint32_t pk[16];
-          uint4 rnd = make_uint4(0, 0, 0, 0);
   #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float x0 = fmaf(s[c * 32 + 2 * e], p.scale_log2, -m_use);
@@ -540,15 +548,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p0 = fast_exp2(x0);
             const float p1 = fast_exp2(x1);
             rs[e & 3] += p0 + p1;
-            if (DROP && C::MW) {
+            if (DROP) {
               const uint32_t mw = mbits[c];
               pk[e] = pack_bf16x2(((mw >> (2 * e)) & 1u) ? p0 : 0.f, ((mw >> (2 * e + 1)) & 1u) ? p1 : 0.f);
-            } else if (DROP) {
-              if ((e & 1) == 0)
-                rnd = philox4x32_10((uint32_t)(col_lo + c * 32 + 2 * e) >> 2, (uint32_t)row,
-                                    (uint32_t)bh, p.drop_off, p.seed_lo, p.seed_hi);
-              const uint32_t w0 = (e & 1) ? rnd.z : rnd.x, w1 = (e & 1) ? rnd.w : rnd.y;
-              pk[e] = pack_bf16x2(w0 >= p.drop_thr ? p0 : 0.f, w1 >= p.drop_thr ? p1 : 0.f);
             } else if constexpr (C::F8) {
               // four e4m3 codes per 32-bit word: keys 2e, 2e + 1 in the low
               // half of word e / 2 for even e, in the high half for odd e
@@ -671,7 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t row = (uint32_t)(U.q_start + r);
       for (int j = 0; j < U.nkb && ok; ++j) {
         const int gj = g + j;
-        ok = warp_wait_all(bar(B_MEMPTY + (gj & 1)), ((gj >> 1) & 1) ^ 1, wc);
+        const int mbuf = gj % C::MASK_NBUF;
+        ok = warp_wait_all(bar(B_MEMPTY + mbuf), ((gj / C::MASK_NBUF) & 1) ^ 1, wc);
         if (!ok) break;
         const uint32_t c0 = (uint32_t)((U.j0 + j) * C::BN) >> 2;
         uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -689,8 +692,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             w[q4] |= nib << (4 * kk);
           }
         }
-        st_shared_v4(sbase + C::OFF_MASK + (gj & 1) * C::MASK_BUF + r * (C::BN / 8), w[0], w[1], w[2], w[3]);
-        mbar_arrive(bar(B_MFULL + (gj & 1)));
+        st_shared_v4(sbase + C::OFF_MASK + mbuf * C::MASK_BUF + r * (C::BN / 8), w[0], w[1], w[2], w[3]);
+        mbar_arrive(bar(B_MFULL + mbuf));
       }
       g += U.nkb;
     }
@@ -750,12 +753,10 @@ int run_fwd(const AttnArgs &a) {
   p.o_scale = a.drop_thr != 0 ? a.drop_scale : (C::F8 ? a.descale_v : 1.f);
   p.err = a.err;
   if (a.drop_thr != 0 && a.splits > 1) return 2;   // dropout only in the plain forward
-  if (a.drop_thr != 0 && !C::MW && C::D != 256) return 2;   // d = 64, 128: the mask-warp instances
+  if (a.drop_thr != 0 && !C::MW) return 2;   // dropout: the mask-warp instances
   // dropout: the mask-warp instances (d = 64, 128) or, at d = 256, the
   // instance whose softmax thread evaluates the mask itself
   auto kern = fwd_kernel<C, C::MW>;
-  if constexpr (!C::F8 && !C::MW && C::D == 256)
-    if (a.drop_thr != 0) kern = fwd_kernel<C, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return 5;
@@ -889,7 +890,9 @@ int launch_fwd_bf16_sm100(const AttnArgs &a) {
     case 128:
       return a.drop_thr && a.splits == 1 ? run_fwd<FwdCfg<128, 1, 128, 2, 2, true>>(a)
                                          : run_fwd<FwdCfg<128, 2, 128, 1, 2>>(a);
-    case 256: return run_fwd<FwdCfg<256, 1, 128, 1, 2>>(a);
+    case 256:
+      return a.drop_thr && a.splits == 1 ? run_fwd<FwdCfg<256, 1, 128, 1, 2, true>>(a)
+                                         : run_fwd<FwdCfg<256, 1, 128, 1, 2>>(a);
     default: return 2;
   }
 }
