@@ -24,7 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libfa.so")
 _lib = None
 
-EXPORTS = ("fa_fwd", "fa_fwd_fp8", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_splitkv",
+EXPORTS = ("fa_fwd", "fa_fwd_pair", "fa_fwd_fp8", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_splitkv",
            "fa_fwd_splitkv_num_splits",
            "fa_fwd_splitkv_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prep",
            "fa_bwd_dkdv",
@@ -50,6 +50,8 @@ def lib():
         dims = [I, I, I, I, I, I, F, I, P]
         L.fa_fwd.argtypes = [P] * 5 + dims
         L.fa_fwd.restype = I
+        L.fa_fwd_pair.argtypes = [P] * 5 + dims
+        L.fa_fwd_pair.restype = I
         L.fa_fwd_f32.argtypes = [P] * 5 + dims
         L.fa_fwd_f32.restype = I
         U64 = ctypes.c_ulonglong
@@ -90,6 +92,10 @@ def lib():
 # ----------------------------------------------------------------- raw ABI
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
     return lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, int(causal), stream)
+
+
+def fa_fwd_pair(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream=0):
+    return lib().fa_fwd_pair(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, int(causal), stream)
 
 
 def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, descale_q, descale_k, descale_v, causal,
@@ -249,9 +255,10 @@ def _stream(t):
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
-def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
+def forward(q, k, v, scale=None, causal=False, out=None, lse=None, cta_pair=False):
     """O, L = attention(q, k, v) for contiguous CUDA tensors [B, H, N, d]
-    (bf16 -> fa_fwd, float32 -> fa_fwd_f32)."""
+    (bf16 -> fa_fwd, or fa_fwd_pair with cta_pair=True; float32 ->
+    fa_fwd_f32)."""
     import torch
     _check_qkv("forward", q, k, v, (torch.bfloat16, torch.float32))
     _check_cuda("forward", q, k, v)
@@ -263,7 +270,9 @@ def forward(q, k, v, scale=None, causal=False, out=None, lse=None):
             or L.dtype != torch.float32):
         raise ValueError("forward: out must be shaped and typed like q, lse float32 [B, Hq, Nq]")
     _check_cuda("forward", q, o, L)
-    fn = fa_fwd if q.dtype == torch.bfloat16 else fa_fwd_f32
+    if cta_pair and q.dtype != torch.bfloat16:
+        raise ValueError("forward: cta_pair=True needs bf16 tensors")
+    fn = (fa_fwd_pair if cta_pair else fa_fwd) if q.dtype == torch.bfloat16 else fa_fwd_f32
     with _on(q):
         _check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), L.data_ptr(), B, Hq, Hkv,
                   Nq, Nk, d, scale, causal, _stream(q)), fn.__name__)

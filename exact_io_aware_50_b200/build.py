@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfa.so")
 SOURCES = ["fa_capi.cu", "fa_simt.cu", "fa_fwd_sm100.cu", "fa_bwd_sm100.cu", "fa_noalloc.cu"]
-HEADERS = ["common.cuh", "launch.h"]
+HEADERS = ["common.cuh", "cta_pair.cuh", "launch.h"]
 
 
 def nvcc() -> str:

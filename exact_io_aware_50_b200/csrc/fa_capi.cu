@@ -166,6 +166,25 @@ FA_EXPORT int fa_fwd(const void *q, const void *k, const void *v, void *o, float
   return fa::launch_fwd_bf16_sm100(a);
 }
 
+FA_EXPORT int fa_fwd_pair(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                          int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                          fa_stream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int st = fa::check_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal);
+  if (st) return st;
+  if (d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!fa::aligned16(q) || !fa::aligned16(k) || !fa::aligned16(v) || !fa::aligned16(o) ||
+      !fa::aligned16(lse))
+    return FA_ERR_ALIGNMENT;
+  AttnArgs a;
+  int dev;
+  if ((st = fa::prologue(&dev, a))) return st;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.d = d;
+  a.scale = scale; a.causal = causal ? 1 : 0; a.stream = (cudaStream_t)stream;
+  return fa::launch_fwd_pair_bf16_sm100(a);
+}
+
 FA_EXPORT int fa_fwd_splitkv_num_splits(int B, int Hq, int Nq, int Nk, int d) {
   if (B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0) return 0;
   if (d != 64 && d != 128 && d != 256) return 0;

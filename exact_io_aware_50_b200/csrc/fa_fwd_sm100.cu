@@ -72,6 +72,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "cta_pair.cuh"
 #include "launch.h"
 
 namespace fa {
@@ -94,10 +95,15 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // key blocks ahead and leave one bit per (query row, key) in a double-
 // buffered array in shared memory, so the softmax thread tests bits instead
 // of evaluating a Philox call per four keys.
-template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2, bool MW_ = false>
+// PAIR: a cluster of two CTAs shares each tile's MMAs (cta_group::2, M =
+// 256): each CTA holds its own NT Q tiles, half of each K tile (64 of the
+// 128 keys) and half of each V tile (D / 2 of the columns), so a K/V ring
+// slot takes half the shared memory and half the load bytes per SM; the even
+// CTA issues the MMAs for both.
+template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2, bool MW_ = false, bool PAIR_ = false>
 struct FwdCfg {
   static constexpr int D = D_, NT = NT_, BN = BN_, STAGES = STAGES_, ES = ES_;
-  static constexpr bool MW = MW_;
+  static constexpr bool MW = MW_, PAIR = PAIR_;
   static constexpr bool F8 = ES == 1;
   static constexpr int DCH = D * ES / 128;                // 128-byte column chunks
   static constexpr int CH_ELEMS = 128 / ES;               // elements per chunk (TMA box width)
@@ -112,15 +118,23 @@ struct FwdCfg {
   static constexpr int Q_CHUNK = BM * 128;                // bytes of one chunk of a Q tile
   static constexpr int KV_CHUNK = BN * 128;
   static constexpr int Q_TILE = Q_CHUNK * DCH;
-  static constexpr int KV_TILE = KV_CHUNK * DCH;
+  // this CTA's share of a K tile (rows) and of a V tile (128-byte column chunks)
+  static constexpr int K_ROWS = PAIR ? BN / 2 : BN;
+  static constexpr int V_DCH = PAIR ? DCH / 2 : DCH;
+  static constexpr int K_CHUNK = K_ROWS * 128;
+  static constexpr int K_TILE = K_CHUNK * DCH;
+  static constexpr int V_TILE = KV_CHUNK * V_DCH;
+  // query rows of one work unit (both CTAs of a pair)
+  static constexpr int UROWS = (PAIR ? 2 : 1) * NT * 128;
+  static constexpr int MMA_M = PAIR ? 256 : 128;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NT * Q_TILE;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
+  static constexpr int OFF_V = OFF_K + STAGES * K_TILE;
   // P tiles: [NT][BM rows][BN * ES bytes], K-major 128-byte swizzled chunks
   static constexpr int P_ROWB = BN * ES;
   static constexpr int P_CHUNK = BM * 128;
   static constexpr int P_TILE = P_CHUNK * (P_ROWB / 128);
-  static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;
+  static constexpr int OFF_P = OFF_V + STAGES * V_TILE;
   static constexpr int MASK_BUF = BM * BN / 8;            // [MASK_NBUF][BM rows][BN bits]
   // d = 256 has room for one mask buffer only (and no alignment slack: the
   // dynamic shared window is 1024-byte aligned, checked at run time)
@@ -145,6 +159,7 @@ struct FwdCfg {
   static_assert(ES == 1 || ES == 2, "bf16 or e4m3 operands");
   static_assert(D * ES % 128 == 0, "whole 128-byte rows per chunk");
   static_assert(!MW || (NT == 1 && ES == 2 && BN == 128), "mask warps: one bf16 tile per CTA");
+  static_assert(!PAIR || (!MW && ES == 2 && DCH % 2 == 0), "pairs: bf16, d = 128 or 256, no dropout");
 };
 
 struct FwdParams {
@@ -194,14 +209,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = warp_id_uniform();
   const int lane = threadIdx.x & 31;
+  // CTA pairs: the pair runs one unit sequence; its rank-0 CTA (the leader)
+  // issues the MMAs and owns the barriers they wait on.
+  const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  // cluster address of the leader's barrier i (pairs)
+  auto lbar = [&](int i) { return mapa_shared(bar(i), 0); };
+  // arrive on a barrier the MMA issuer waits for
+  auto arrive_mma = [&](int i) {
+    if constexpr (C::PAIR) mbar_arrive_cluster(lbar(i));
+    else mbar_arrive(bar(i));
+  };
 
-  // Persistent CTAs: round k gives CTA c unit k*G + c (k even) or
-  // k*G + G-1-c (k odd), G = gridDim.x.  Unit order:
+  // Persistent CTAs (or pairs): round k gives CTA c unit k*G + c (k even)
+  // or k*G + G-1-c (k odd), G = gridDim.x (pairs: G pairs, c the pair's
+  // index).  Unit order:
   // causal, the heaviest query blocks of every head first; otherwise head by
   // head, so the K and V tiles a wave reads are those of a few heads and stay
   // in L2.  Split-KV: the piece index is the slowest-varying part.
   const int per_piece = p.nqb * p.BH;
   const int total_units = per_piece * p.splits;
+  const int G = (int)gridDim.x / (C::PAIR ? 2 : 1);
+  const int cid = (int)blockIdx.x / (C::PAIR ? 2 : 1);
+  auto unit_at = [&](int k) { return k * G + ((k & 1) ? G - 1 - cid : cid); };
   struct Unit {
     int piece, bh, bh_kv, q_start, j0, nkb;
   };
@@ -213,10 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     U.bh = p.causal ? v % p.BH : v / p.nqb;
     const int b = U.bh / p.Hq, h = U.bh % p.Hq;
     U.bh_kv = b * p.Hkv + h / (p.Hq / p.Hkv);
-    U.q_start = qblk * C::NT * BM;
+    U.q_start = qblk * C::UROWS;
     const int nkb_all = (p.Nk + C::BN - 1) / C::BN;
     const int nkb_vis = p.causal
-                            ? min(nkb_all, (U.q_start + C::NT * BM + p.causal_off + C::BN - 1) / C::BN)
+                            ? min(nkb_all, (U.q_start + C::UROWS + p.causal_off + C::BN - 1) / C::BN)
                             : nkb_all;
     // key blocks [j0, j0 + nkb) of this piece
     const int per_split = (nkb_vis + p.splits - 1) / p.splits;
@@ -224,6 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     U.nkb = min(nkb_vis, U.j0 + per_split) - U.j0;
     return U;
   };
+  // first query row of this CTA's tile t of unit U
+  auto tile_row0 = [&](const Unit &U, int t) { return U.q_start + ((int)rank * C::NT + t) * BM; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -236,10 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < C::NT; ++t) {
       mbar_init(bar(B_SFULL + t), 1);
-      mbar_init(bar(B_PFULL + t), BM);
+      // arrivals of the softmax threads: both CTAs' in a pair
+      mbar_init(bar(B_PFULL + t), (C::PAIR ? 2 : 1) * BM);
       mbar_init(bar(B_OFULL + t), 1);
-      mbar_init(bar(B_OEMPTY + t), BM);
-      mbar_init(bar(B_SEMPTY + t), BM);
+      mbar_init(bar(B_OEMPTY + t), (C::PAIR ? 2 : 1) * BM);
+      mbar_init(bar(B_SEMPTY + t), (C::PAIR ? 2 : 1) * BM);
       mbar_init(bar(B_PEMPTY + t), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
@@ -251,8 +284,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), C::TM_ALLOC);
-    tmem_relinquish();
+    // pairs: warp 0 of both CTAs allocates the same columns in each
+    if constexpr (C::PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), C::TM_ALLOC);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), C::TM_ALLOC);
+      tmem_relinquish();
+    }
   }
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmQ);
@@ -260,7 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmV);
   }
   tc_fence_before();
-  __syncthreads();
+  // pairs: the peer's first arrivals on the leader's barriers come after this
+  if constexpr (C::PAIR) cluster_sync_all();
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   WaitCtx wc{p.err, abort_flag, kWaitLimitNs};
@@ -276,42 +317,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last_q_phase = -1;
       bool ok = true;
       int g = 0, uq = 0;
-      for (int k = 0; ok && k * (int)gridDim.x < total_units; ++k) {
+      // A tile load completing on full-barrier fb: pairs load this CTA's half
+      // and complete on the leader's barrier, where the leader alone has
+      // announced both halves' bytes.
+      auto load = [&](uint32_t dst, const CUtensorMap *m, int fb, int c0, int c1, int c2) {
+        if constexpr (C::PAIR) tma_load_3d_pair(dst, m, lbar(fb), c0, c1, c2);
+        else tma_load_3d(dst, m, bar(fb), c0, c1, c2);
+      };
+      constexpr uint32_t HALVES = C::PAIR ? 2 : 1;
+      for (int k = 0; ok && k * G < total_units; ++k) {
         // snake order: even rounds ascending, odd rounds descending, so the
         // heavy-first unit list pairs heavy with light units on each CTA
-        const int u = k * (int)gridDim.x +
-                      ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+        const int u = unit_at(k);
         if (u >= total_units) continue;
         const Unit U = decode(u);
         if (U.nkb == 0) continue;
         // the previous unit's S MMAs must be done with the Q tiles
         ok = bounded_wait(bar(B_QEMPTY), (uq & 1) ^ 1, wc);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(B_QFULL), C::NT * C::Q_TILE);
+        if (leader) mbar_arrive_expect_tx(bar(B_QFULL), HALVES * C::NT * C::Q_TILE);
         for (int t = 0; t < C::NT; ++t)
           for (int c = 0; c < C::DCH; ++c)
-            tma_load_3d(sbase + C::OFF_Q + t * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(B_QFULL),
-                        c * C::CH_ELEMS, U.q_start + t * BM, U.bh);
+            load(sbase + C::OFF_Q + t * C::Q_TILE + c * C::Q_CHUNK, &tmQ, B_QFULL,
+                 c * C::CH_ELEMS, tile_row0(U, t), U.bh);
         last_q_phase = uq & 1;
+        // K: this CTA's K_ROWS keys of the block, all columns
         auto load_k = [&](int j) {
           const int s = (g + j) % C::STAGES;
           const uint32_t ph = ((g + j) / C::STAGES) & 1;
           if (!bounded_wait(bar(B_KEMPTY + s), ph ^ 1, wc)) return false;
-          mbar_arrive_expect_tx(bar(B_KFULL + s), C::KV_TILE);
+          if (leader) mbar_arrive_expect_tx(bar(B_KFULL + s), HALVES * C::K_TILE);
           for (int c = 0; c < C::DCH; ++c)
-            tma_load_3d(sbase + C::OFF_K + s * C::KV_TILE + c * C::KV_CHUNK, &tmK,
-                        bar(B_KFULL + s), c * C::CH_ELEMS, (U.j0 + j) * C::BN, U.bh_kv);
+            load(sbase + C::OFF_K + s * C::K_TILE + c * C::K_CHUNK, &tmK, B_KFULL + s,
+                 c * C::CH_ELEMS, (U.j0 + j) * C::BN + (int)rank * C::K_ROWS, U.bh_kv);
           last_k_phase[s] = ph;
           return true;
         };
+        // V: all keys of the block, this CTA's V_DCH column chunks
         auto load_v = [&](int j) {
           const int s = (g + j) % C::STAGES;
           const uint32_t ph = ((g + j) / C::STAGES) & 1;
           if (!bounded_wait(bar(B_VEMPTY + s), ph ^ 1, wc)) return false;
-          mbar_arrive_expect_tx(bar(B_VFULL + s), C::KV_TILE);
-          for (int c = 0; c < C::DCH; ++c)
-            tma_load_3d(sbase + C::OFF_V + s * C::KV_TILE + c * C::KV_CHUNK, &tmV,
-                        bar(B_VFULL + s), c * C::CH_ELEMS, (U.j0 + j) * C::BN, U.bh_kv);
+          if (leader) mbar_arrive_expect_tx(bar(B_VFULL + s), HALVES * C::V_TILE);
+          for (int c = 0; c < C::V_DCH; ++c)
+            load(sbase + C::OFF_V + s * C::V_TILE + c * C::KV_CHUNK, &tmV, B_VFULL + s,
+                 ((int)rank * C::V_DCH + c) * C::CH_ELEMS, (U.j0 + j) * C::BN, U.bh_kv);
           last_v_phase[s] = ph;
           return true;
         };
@@ -325,8 +375,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         g += U.nkb;
         ++uq;
       }
-      if (!ok) {
+      if (!ok && leader) {
         // Drain: let every copy this role issued land before the CTA exits.
+        // (A pair's copies complete on the leader's barriers: the leader
+        // drains them, the peer cannot observe its own.)
         if (last_q_phase >= 0) (void)drain_wait(bar(B_QFULL), last_q_phase, p.err, kWaitLimitNs);
         for (int s = 0; s < C::STAGES; ++s) {
           if (last_k_phase[s] >= 0) (void)drain_wait(bar(B_KFULL + s), last_k_phase[s], p.err, kWaitLimitNs);
@@ -337,30 +389,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t IDESC_S = C::F8 ? idesc_e4m3(BM, C::BN, 0, 0) : idesc_bf16(BM, C::BN, 0, 0);
-    constexpr uint32_t IDESC_PV = C::F8 ? idesc_e4m3(BM, C::D, 0, 1) : idesc_bf16(BM, C::D, 0, 1);
+    // pairs: M = 256 (each CTA's 128 rows), N the whole block / head dim
+    constexpr uint32_t IDESC_S =
+        C::F8 ? idesc_e4m3(BM, C::BN, 0, 0) : idesc_bf16(C::MMA_M, C::BN, 0, 0);
+    constexpr uint32_t IDESC_PV =
+        C::F8 ? idesc_e4m3(BM, C::D, 0, 1) : idesc_bf16(C::MMA_M, C::D, 0, 1);
+    auto mma16 = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+      if constexpr (C::PAIR) mma_ss_pair(d, a, b, idesc, acc);
+      else mma_ss(d, a, b, idesc, acc);
+    };
+    // MMA completion: pairs arrive on the barrier in both CTAs
+    auto commit = [&](int i) {
+      if constexpr (C::PAIR) mma_commit_pair_both(bar(i));
+      else mma_commit(bar(i));
+    };
+    // barriers the peer's threads arrive on (pairs) need cluster-scope acquire
+    auto wait = [&](int i, uint32_t ph) {
+      if constexpr (C::PAIR) return bounded_wait_cluster(bar(i), ph, wc);
+      else return bounded_wait(bar(i), ph, wc);
+    };
     // Descriptors are built once; each MMA offsets a base descriptor.
     const uint64_t dq0 = sw128_desc(sbase + C::OFF_Q, 16, 1024);
     const uint64_t dk0 = sw128_desc(sbase + C::OFF_K, 16, 1024);
     const uint64_t dv0 = sw128_desc(sbase + C::OFF_V, C::KV_CHUNK, 1024);
     auto issue_S = [&](int t, int s) {
       const uint64_t qa = desc_add(dq0, t * C::Q_TILE);
-      const uint64_t kb = desc_add(dk0, s * C::KV_TILE);
+      const uint64_t kb = desc_add(dk0, s * C::K_TILE);
 #pragma unroll
       for (int kk = 0; kk < C::S_STEPS; ++kk) {
         const uint32_t off = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
-        const uint32_t offk = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
+        const uint32_t offk = (kk >> 2) * C::K_CHUNK + (kk & 3) * 32;
         if constexpr (C::F8)
           mma_ss_f8(tmem + C::TM_S + t * C::BN, desc_add(qa, off), desc_add(kb, offk), IDESC_S,
                     kk > 0);
         else
-          mma_ss(tmem + C::TM_S + t * C::BN, desc_add(qa, off), desc_add(kb, offk), IDESC_S,
-                 kk > 0);
+          mma16(tmem + C::TM_S + t * C::BN, desc_add(qa, off), desc_add(kb, offk), IDESC_S,
+                kk > 0);
       }
     };
     const uint64_t dp0 = sw128_desc(sbase + C::OFF_P, 16, 1024);
     auto issue_PV = [&](int t, int s, bool first) {
-      const uint64_t vb = desc_add(dv0, s * C::KV_TILE);
+      const uint64_t vb = desc_add(dv0, s * C::V_TILE);
       const uint64_t pa = desc_add(dp0, t * C::P_TILE);
 #pragma unroll
       for (int kk = 0; kk < C::PV_STEPS; ++kk) {
@@ -371,32 +440,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss_f8(tmem + C::TM_O + t * C::D, desc_add(pa, offp), desc_add(vb, kk * C::MMA_K * 128),
                     IDESC_PV, (!first) || kk > 0);
         else
-          mma_ss(tmem + C::TM_O + t * C::D, desc_add(pa, offp), desc_add(vb, kk * C::MMA_K * 128),
-                 IDESC_PV, (!first) || kk > 0);
+          mma16(tmem + C::TM_O + t * C::D, desc_add(pa, offp), desc_add(vb, kk * C::MMA_K * 128),
+                IDESC_PV, (!first) || kk > 0);
       }
     };
-    // The whole role runs in lane 0; the other lanes wait at the end.
-    if (lane == 0) {
+    // The whole role runs in lane 0 (of the leader, in a pair); the other
+    // lanes wait at the end.
+    if (lane == 0 && leader) {
       bool ok = true;
       int g = 0, uq = 0;
-      for (int k = 0; ok && k * (int)gridDim.x < total_units; ++k) {
+      for (int k = 0; ok && k * G < total_units; ++k) {
         // snake order: even rounds ascending, odd rounds descending, so the
         // heavy-first unit list pairs heavy with light units on each CTA
-        const int u = k * (int)gridDim.x +
-                      ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+        const int u = unit_at(k);
         if (u >= total_units) continue;
         const Unit U = decode(u);
         if (U.nkb == 0) continue;
-        ok = bounded_wait(bar(B_QFULL), uq & 1, wc);
-        if (ok) ok = bounded_wait(bar(B_KFULL + g % C::STAGES), (g / C::STAGES) & 1, wc);
+        ok = wait(B_QFULL, uq & 1);
+        if (ok) ok = wait(B_KFULL + g % C::STAGES, (g / C::STAGES) & 1);
         if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < C::NT; ++t) {
           issue_S(t, g % C::STAGES);
-          mma_commit(bar(B_SFULL + t));
+          commit(B_SFULL + t);
         }
-        mma_commit(bar(B_KEMPTY + g % C::STAGES));
-        if (U.nkb == 1) mma_commit(bar(B_QEMPTY));   // last S of the unit issued
+        commit(B_KEMPTY + g % C::STAGES);
+        if (U.nkb == 1) commit(B_QEMPTY);   // last S of the unit issued
         // S_t(j+1) as soon as the softmax has read S_t(j); P_t(j) V_j once
         // P_t(j) is in shared memory.
         for (int j = 0; j < U.nkb && ok; ++j) {
@@ -405,37 +474,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = (gj / C::STAGES) & 1;
           if (j + 1 < U.nkb) {
             const int s1 = (gj + 1) % C::STAGES;
-            ok = bounded_wait(bar(B_KFULL + s1), ((gj + 1) / C::STAGES) & 1, wc);
+            ok = wait(B_KFULL + s1, ((gj + 1) / C::STAGES) & 1);
             for (int t = 0; t < C::NT && ok; ++t) {
-              ok = bounded_wait(bar(B_SEMPTY + t), gj & 1, wc);
+              ok = wait(B_SEMPTY + t, gj & 1);
               if (!ok) break;
               tc_fence_after();
               issue_S(t, s1);
-              mma_commit(bar(B_SFULL + t));
+              commit(B_SFULL + t);
             }
             if (!ok) break;
-            mma_commit(bar(B_KEMPTY + s1));
-            if (j + 2 == U.nkb) mma_commit(bar(B_QEMPTY));   // last S of the unit
+            commit(B_KEMPTY + s1);
+            if (j + 2 == U.nkb) commit(B_QEMPTY);   // last S of the unit
           }
-          ok = bounded_wait(bar(B_VFULL + s), ph, wc);
+          ok = wait(B_VFULL + s, ph);
           for (int t = 0; t < C::NT && ok; ++t) {
-            ok = bounded_wait(bar(B_PFULL + t), gj & 1, wc);
+            ok = wait(B_PFULL + t, gj & 1);
             if (ok && j == 0 && uq > 0)   // the previous unit's epilogue has read O_t
-              ok = bounded_wait(bar(B_OEMPTY + t), (uq - 1) & 1, wc);
+              ok = wait(B_OEMPTY + t, (uq - 1) & 1);
             if (!ok) break;
             tc_fence_after();
             issue_PV(t, s, j == 0);
-            mma_commit(bar(B_PEMPTY + t));
-            if (j + 1 == U.nkb) mma_commit(bar(B_OFULL + t));
+            commit(B_PEMPTY + t);
+            if (j + 1 == U.nkb) commit(B_OFULL + t);
           }
-          if (ok) mma_commit(bar(B_VEMPTY + s));
+          if (ok) commit(B_VEMPTY + s);
         }
         g += U.nkb;
         ++uq;
       }
       if (!ok) {
         // Drain: every MMA issued so far must finish before TMEM is freed.
-        mma_commit(bar(B_DRAIN));
+        if constexpr (C::PAIR) mma_commit_pair_local(bar(B_DRAIN));
+        else mma_commit(bar(B_DRAIN));
         (void)drain_wait(bar(B_DRAIN), 0, p.err, kWaitLimitNs);
       }
     }
@@ -449,15 +519,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_off + C::TM_O + t * C::D;
     bool ok = true;
     int g = 0, uq = 0;
-    for (int k = 0; ok && k * (int)gridDim.x < total_units; ++k) {
+    for (int k = 0; ok && k * G < total_units; ++k) {
         // snake order: even rounds ascending, odd rounds descending, so the
         // heavy-first unit list pairs heavy with light units on each CTA
-        const int u = k * (int)gridDim.x +
-                      ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+        const int u = unit_at(k);
         if (u >= total_units) continue;
       const Unit U = decode(u);
       const int bh = U.bh;
-      const int row = U.q_start + t * BM + r;     // query row
+      const int row = tile_row0(U, t) + r;     // query row
       if (U.nkb == 0) {
         // An empty piece (only in split mode): its rows see no key here.
         if (row < p.Nq) {
@@ -468,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         continue;
       }
-      const int row_lo = U.q_start + t * BM;
+      const int row_lo = tile_row0(U, t);
       // keys [0, limit) visible
       const int limit_row = p.causal ? min(p.Nk, row + 1 + p.causal_off) : p.Nk;
       float m_run = -INFINITY, l_run = 0.f;
@@ -483,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         // S_t is in registers: its TMEM columns may take S_t(j+1)
         tc_fence_before();
-        mbar_arrive(bar(B_SEMPTY + t));
+        arrive_mma(B_SEMPTY + t);
         float *s = reinterpret_cast<float *>(sr);
         const int col_lo = (U.j0 + j) * C::BN;
         // dropout with mask warps: bit 32 c + b of this row's 128 = key
@@ -593,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL + t));
+        arrive_mma(B_PFULL + t);
       }
       // ---------------------------------------------------------- epilogue
       if (ok) ok = warp_wait_all(bar(B_OFULL + t), uq & 1, wc);
@@ -621,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(bar(B_OEMPTY + t));   // O_t read out: the next unit may overwrite it
+        arrive_mma(B_OEMPTY + t);   // O_t read out: the next unit may overwrite it
         if (live)
           p.l_part[prow] =
               empty ? -INFINITY : (m_run + __log2f(l_run) - C::P_SHIFT) * 0.69314718055994531f;
@@ -648,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(bar(B_OEMPTY + t));   // O_t read out: the next unit may overwrite it
+        arrive_mma(B_OEMPTY + t);   // O_t read out: the next unit may overwrite it
         if (live)
           p.o_lse[(size_t)bh * p.Nq + row] =
               (m_run + __log2f(l_run) - C::P_SHIFT) * 0.69314718055994531f;
@@ -665,9 +734,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = threadIdx.x - 4 * 32;
     bool ok = true;
     int g = 0;
-    for (int k = 0; ok && k * (int)gridDim.x < total_units; ++k) {
-      const int u = k * (int)gridDim.x +
-                    ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    for (int k = 0; ok && k * G < total_units; ++k) {
+      const int u = unit_at(k);
       if (u >= total_units) continue;
       const Unit U = decode(u);
       const uint32_t row = (uint32_t)(U.q_start + r);
@@ -700,10 +768,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  // pairs: neither CTA leaves (or frees its TMEM) while the other may still
+  // arrive on its barriers or the leader's MMAs may still use it
+  if constexpr (C::PAIR) cluster_sync_all();
+  else __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TM_ALLOC);
+    if constexpr (C::PAIR) tmem_dealloc_pair(tmem, C::TM_ALLOC);
+    else tmem_dealloc(tmem, C::TM_ALLOC);
   }
 }
 
@@ -728,14 +800,14 @@ int run_fwd(const AttnArgs &a) {
   CUtensorMap mq, mk, mv;
   if (C::F8 && (a.drop_thr != 0 || a.splits > 1)) return 2;   // e4m3: plain forward only
   if (!make_map(&mq, a.q, a.Nq, a.B * a.Hq, C::D, BM, C::ES) ||
-      !make_map(&mk, a.k, a.Nk, a.B * a.Hkv, C::D, C::BN, C::ES) ||
+      !make_map(&mk, a.k, a.Nk, a.B * a.Hkv, C::D, C::K_ROWS, C::ES) ||
       !make_map(&mv, a.v, a.Nk, a.B * a.Hkv, C::D, C::BN, C::ES))
     return 5;
   FwdParams p;
   p.o_lse = a.lse;
   p.o = (__nv_bfloat16 *)a.o;
   p.Hq = a.Hq; p.Hkv = a.Hkv; p.Nq = a.Nq; p.Nk = a.Nk;
-  p.nqb = (a.Nq + C::NT * BM - 1) / (C::NT * BM);
+  p.nqb = (a.Nq + C::UROWS - 1) / C::UROWS;
   p.BH = a.B * a.Hq;
   // e4m3: the Q and K descales fold into the score scale
   p.scale_log2 = (float)((double)a.scale * (C::F8 ? (double)a.descale_q * a.descale_k : 1.0) *
@@ -754,8 +826,7 @@ int run_fwd(const AttnArgs &a) {
   p.err = a.err;
   if (a.drop_thr != 0 && a.splits > 1) return 2;   // dropout only in the plain forward
   if (a.drop_thr != 0 && !C::MW) return 2;   // dropout: the mask-warp instances
-  // dropout: the mask-warp instances (d = 64, 128) or, at d = 256, the
-  // instance whose softmax thread evaluates the mask itself
+  if (C::PAIR && a.splits > 1) return 2;      // pairs: plain forward only
   auto kern = fwd_kernel<C, C::MW>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
@@ -766,6 +837,28 @@ int run_fwd(const AttnArgs &a) {
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return 5;
+  if constexpr (C::PAIR) {
+    // clusters of two CTAs, one pair per unit up to the number of pairs
+    // that fit at once
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = a.stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)(2 * (sms / 2)), 1, 1);
+    int pairs = 0;
+    if (cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg) != cudaSuccess || pairs < 1) return 5;
+    const long long npairs = units < pairs ? units : pairs;
+    cfg.gridDim = dim3((unsigned)(2 * npairs), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p) != cudaSuccess) return 5;
+    return cudaGetLastError() == cudaSuccess ? 0 : 5;
+  }
   const long long grid = units < sms ? units : sms;
   kern<<<(unsigned)grid, kThreads, C::SMEM, a.stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : 5;
@@ -876,6 +969,16 @@ int launch_fwd_e4m3_sm100(const AttnArgs &a) {
   switch (a.d) {
     case 128: return run_fwd<FwdCfg<128, 2, 128, 3, 1>>(a);
     case 256: return run_fwd<FwdCfg<256, 1, 128, 2, 1>>(a);
+    default: return 2;
+  }
+}
+
+// CTA-pair forward (bf16, no dropout, plain forward): d = 128 and 256.
+int launch_fwd_pair_bf16_sm100(const AttnArgs &a) {
+  if (a.drop_thr != 0 || a.splits > 1) return 2;
+  switch (a.d) {
+    case 128: return run_fwd<FwdCfg<128, 2, 128, 3, 2, false, true>>(a);
+    case 256: return run_fwd<FwdCfg<256, 1, 128, 2, 2, false, true>>(a);
     default: return 2;
   }
 }

@@ -69,6 +69,7 @@ int launch_fwd_f32(const AttnArgs &a);
 int launch_bwd_f32(const AttnArgs &a);
 int launch_fwd_bf16_sm100(const AttnArgs &a);
 int launch_fwd_splitkv_bf16_sm100(const AttnArgs &a);   // pieces + merge (splits > 1)
+int launch_fwd_pair_bf16_sm100(const AttnArgs &a);      // CTA-pair form (d = 128, 256)
 int launch_fwd_e4m3_sm100(const AttnArgs &a);   // e4m3 Q/K/V, bf16 O (d = 128, 256)
 int launch_bwd_bf16_sm100(const AttnArgs &a);   // all three stages
 int launch_bwd_prep_bf16(const AttnArgs &a);     // D + zeroed dQ accumulator

@@ -73,6 +73,21 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
            fa_stream_t stream);
 
 /*
+ * fa_fwd_pair -- fa_fwd computed by pairs of CTAs on neighbouring SMs that
+ * share each tile's tensor-core MMAs (tcgen05 cta_group::2, M = 256: the
+ * two-CTA MMA the wiki's FlashAttention-4 paragraph lists).  Each CTA of a
+ * pair holds its own 128-row Q tiles and loads half of every K tile (64 of
+ * the 128 keys) and half of every V tile (d / 2 of the columns), so a pair
+ * moves each K/V block into shared memory once instead of twice.  Same
+ * arguments, layouts, result and errors as fa_fwd; d must be 128 or 256
+ * (FA_ERR_UNSUPPORTED otherwise).  fa_fwd itself uses the single-CTA
+ * kernels, measured faster on B200 for the shapes it is timed on.
+ */
+int fa_fwd_pair(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                fa_stream_t stream);
+
+/*
  * Split-KV forward for inference shapes -- few query rows per head against a
  * long key range (the FlashAttention blog, section 4.2, on batch-1 inference
  * leaving the GPU idle when only batch and heads are parallel).  The visible

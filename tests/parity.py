@@ -85,13 +85,13 @@ def f64(t):
 
 
 def run_full_check(B, Hq, Hkv, Nq, Nk, d, causal, dtype="bf16", seed=0, q_mul=1.0, k_add=0.0,
-                   backward=True, scale=None):
+                   backward=True, scale=None, cta_pair=False):
     """Whole-tensor parity of forward (and backward) against the oracle."""
     dt = torch.bfloat16 if dtype == "bf16" else torch.float32
     x = attn_inputs.draw(B, Hq, Hkv, Nq, Nk, d, seed, dt, q_mul, k_add)
     scale = d ** -0.5 if scale is None else scale
     g = to_dev(x)
-    o, lse = F.forward(g["q"], g["k"], g["v"], scale, causal)
+    o, lse = F.forward(g["q"], g["k"], g["v"], scale, causal, cta_pair=cta_pair)
     torch.cuda.synchronize()
     assert F.fa_device_status() == F.FA_OK
     q, k, v, do = (f64(x[n]) for n in ("q", "k", "v", "do"))
