@@ -720,8 +720,8 @@ def load_traffic(workload, kernel):
 
 # The sources each recorded kernel is compiled from.
 KERNEL_SOURCES = {
-    "fa_fwd": ("common.cuh", "fa_fwd_sm100.cu", "launch.h"),
-    "fa_fwd_fp8": ("common.cuh", "fa_fwd_sm100.cu", "launch.h"),
+    "fa_fwd": ("common.cuh", "cta_pair.cuh", "fa_fwd_sm100.cu", "launch.h"),
+    "fa_fwd_fp8": ("common.cuh", "cta_pair.cuh", "fa_fwd_sm100.cu", "launch.h"),
     "fa_bwd_dkdv": ("common.cuh", "fa_bwd_sm100.cu", "launch.h"),
 }
 
