@@ -48,6 +48,16 @@
 // on B200 against the two-tile kernel whose softmax thread evaluated them
 // (causal B4 H16 N4096 d128, p = 0.1): 0.80 -> 0.73 ms.
 //
+// CTA-pair instances (C::PAIR, fa_fwd_pair): clusters of two CTAs on one TPC
+// run one unit sequence; the even CTA issues tcgen05 cta_group::2 MMAs (M =
+// 256) for both, each CTA holding its own Q tiles, 64 of each K block's 128
+// keys and d / 2 of each V block's columns (the two-CTA MMA that the wiki's
+// FlashAttention-4 paragraph lists).  Loads of both CTAs complete on the
+// leader's barriers, MMA commits arrive on both CTAs', and the softmax
+// threads of both arrive on the leader's.  Measured on B200 20-35% slower
+// than the single-CTA instances at d = 128 and 256 (the pair ties the two
+// CTAs' per-block hand-offs together), so fa_fwd does not use it.
+//
 // E4M3 instances (C::F8): Q, K, V are one-byte OCP E4M3 codes with one
 // dequantisation factor each.  S = Q K^T runs as tcgen05 kind::f8f6f4 (K = 32
 // per instruction), the Q and K factors fold into the softmax scale, P is
