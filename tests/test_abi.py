@@ -62,10 +62,11 @@ def test_workspace_size():
 FAKE = 1 << 20  # 16-byte aligned non-null address; never dereferenced (rejected first)
 
 
-@pytest.mark.parametrize("fn", ["fa_fwd", "fa_fwd_f32"])
+@pytest.mark.parametrize("fn", ["fa_fwd", "fa_fwd_f32", "fa_fwd_pair"])
 def test_forward_argument_errors(fn):
     f = getattr(F, fn)
-    ok = dict(B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=64, scale=0.125, causal=0)
+    ok = dict(B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=128 if fn == "fa_fwd_pair" else 64, scale=0.125,
+              causal=0)
 
     def call(ptrs=(FAKE,) * 5, **kw):
         a = dict(ok)
@@ -83,6 +84,9 @@ def test_forward_argument_errors(fn):
     if fn == "fa_fwd":
         assert call(d=96) == F.FA_ERR_UNSUPPORTED
         assert call(d=32) == F.FA_ERR_UNSUPPORTED
+    elif fn == "fa_fwd_pair":
+        assert call(d=64) == F.FA_ERR_UNSUPPORTED   # pairs split d in two 128-byte halves
+        assert call(d=96) == F.FA_ERR_UNSUPPORTED
     else:
         assert call(d=260) == F.FA_ERR_UNSUPPORTED
         assert call(d=6) == F.FA_ERR_UNSUPPORTED
