@@ -110,10 +110,18 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // 128 keys) and half of each V tile (D / 2 of the columns), so a K/V ring
 // slot takes half the shared memory and half the load bytes per SM; the even
 // CTA issues the MMAs for both.
-template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2, bool MW_ = false, bool PAIR_ = false>
+// CSKIP (causal instances with two tiles, whole key range): a unit's last key
+// block lies past tile 0's diagonal, so tile 0 stops one block early (its S
+// and P V for that block are not issued; the block would only add zeros).
+// Used up to 2048 keys: measured on B200 (d = 64 and 128) it gains 10-11% at
+// 512 keys and 1-3% at 2048, is neutral at 4096 and loses 1-4% at 8192 and
+// 16384, where tile 0 running a block ahead into the next unit offsets the
+// two tiles' softmax phases.
+template <int D_, int NT_, int BN_, int STAGES_, int ES_ = 2, bool MW_ = false, bool PAIR_ = false,
+          bool CSKIP_ = false>
 struct FwdCfg {
   static constexpr int D = D_, NT = NT_, BN = BN_, STAGES = STAGES_, ES = ES_;
-  static constexpr bool MW = MW_, PAIR = PAIR_;
+  static constexpr bool MW = MW_, PAIR = PAIR_, CSKIP = CSKIP_;
   static constexpr bool F8 = ES == 1;
   static constexpr int DCH = D * ES / 128;                // 128-byte column chunks
   static constexpr int CH_ELEMS = 128 / ES;               // elements per chunk (TMA box width)
@@ -170,6 +178,7 @@ struct FwdCfg {
   static_assert(D * ES % 128 == 0, "whole 128-byte rows per chunk");
   static_assert(!MW || (NT == 1 && ES == 2 && BN == 128), "mask warps: one bf16 tile per CTA");
   static_assert(!PAIR || (!MW && ES == 2 && DCH % 2 == 0), "pairs: bf16, d = 128 or 256, no dropout");
+  static_assert(!CSKIP || (NT == 2 && !PAIR && !MW), "tile-0 early stop: two tiles per CTA");
 };
 
 struct FwdParams {
@@ -244,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto unit_at = [&](int k) { return k * G + ((k & 1) ? G - 1 - cid : cid); };
   struct Unit {
     int piece, bh, bh_kv, q_start, j0, nkb;
+    int nkb0;   // key blocks of Q tile 0 (CSKIP: one fewer when its diagonal ends earlier)
   };
   auto decode = [&](int u) {
     Unit U;
@@ -262,8 +272,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int per_split = (nkb_vis + p.splits - 1) / p.splits;
     U.j0 = min(nkb_vis, U.piece * per_split);
     U.nkb = min(nkb_vis, U.j0 + per_split) - U.j0;
+    U.nkb0 = U.nkb;
+    if constexpr (C::CSKIP)   // causal, one piece (the launcher checks)
+      U.nkb0 = min(U.nkb, (U.q_start + BM + p.causal_off + C::BN - 1) / C::BN);
     return U;
   };
+  auto nkb_of = [&](const Unit &U, int t) { return (C::CSKIP && t == 0) ? U.nkb0 : U.nkb; };
   // first query row of this CTA's tile t of unit U
   auto tile_row0 = [&](const Unit &U, int t) { return U.q_start + ((int)rank * C::NT + t) * BM; };
 
@@ -459,6 +473,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && leader) {
       bool ok = true;
       int g = 0, uq = 0;
+      // CSKIP: key blocks each tile has processed (its barriers' phases)
+      int gt[C::NT];
+      for (int t = 0; t < C::NT; ++t) gt[t] = 0;
+      auto tile_phase = [&](int t, int j) {
+        return (uint32_t)((C::CSKIP ? gt[t] + j : g + j) & 1);
+      };
       for (int k = 0; ok && k * G < total_units; ++k) {
         // snake order: even rounds ascending, odd rounds descending, so the
         // heavy-first unit list pairs heavy with light units on each CTA
@@ -486,7 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s1 = (gj + 1) % C::STAGES;
             ok = wait(B_KFULL + s1, ((gj + 1) / C::STAGES) & 1);
             for (int t = 0; t < C::NT && ok; ++t) {
-              ok = wait(B_SEMPTY + t, gj & 1);
+              if (C::CSKIP && j + 1 >= nkb_of(U, t)) continue;
+              ok = wait(B_SEMPTY + t, tile_phase(t, j));
               if (!ok) break;
               tc_fence_after();
               issue_S(t, s1);
@@ -498,18 +519,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ok = wait(B_VFULL + s, ph);
           for (int t = 0; t < C::NT && ok; ++t) {
-            ok = wait(B_PFULL + t, gj & 1);
+            if (C::CSKIP && j >= nkb_of(U, t)) continue;
+            ok = wait(B_PFULL + t, tile_phase(t, j));
             if (ok && j == 0 && uq > 0)   // the previous unit's epilogue has read O_t
               ok = wait(B_OEMPTY + t, (uq - 1) & 1);
             if (!ok) break;
             tc_fence_after();
             issue_PV(t, s, j == 0);
             commit(B_PEMPTY + t);
-            if (j + 1 == U.nkb) commit(B_OFULL + t);
+            if (j + 1 == nkb_of(U, t)) commit(B_OFULL + t);
           }
           if (ok) commit(B_VEMPTY + s);
         }
         g += U.nkb;
+        if constexpr (C::CSKIP)
+          for (int t = 0; t < C::NT; ++t) gt[t] += nkb_of(U, t);
         ++uq;
       }
       if (!ok) {
@@ -548,10 +572,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const int row_lo = tile_row0(U, t);
+      const int nkb_t = nkb_of(U, t);   // g counts this tile's key blocks
       // keys [0, limit) visible
       const int limit_row = p.causal ? min(p.Nk, row + 1 + p.causal_off) : p.Nk;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int j = 0; j < U.nkb; ++j) {
+      for (int j = 0; j < nkb_t; ++j) {
         ok = warp_wait_all(bar(B_SFULL + t), (g + j) & 1, wc);
         if (!ok) break;
         tc_fence_after();
@@ -732,7 +757,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.o_lse[(size_t)bh * p.Nq + row] =
               (m_run + __log2f(l_run) - C::P_SHIFT) * 0.69314718055994531f;
       }
-      g += U.nkb;
+      g += nkb_t;
       ++uq;
     }
   } else if (C::MW && warp < 8) {
@@ -837,6 +862,7 @@ int run_fwd(const AttnArgs &a) {
   if (a.drop_thr != 0 && a.splits > 1) return 2;   // dropout only in the plain forward
   if (a.drop_thr != 0 && !C::MW) return 2;   // dropout: the mask-warp instances
   if (C::PAIR && a.splits > 1) return 2;      // pairs: plain forward only
+  if (C::CSKIP && !(a.causal && a.splits == 1)) return 2;
   auto kern = fwd_kernel<C, C::MW>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
@@ -975,9 +1001,15 @@ int launch_fwd_splitkv_bf16_sm100(const AttnArgs &a) {
   }
 }
 
+// Causal with one piece and at most this many keys: tile 0 stops early (CSKIP).
+constexpr int kCskipMaxKeys = 2048;
+
 int launch_fwd_e4m3_sm100(const AttnArgs &a) {
   switch (a.d) {
-    case 128: return run_fwd<FwdCfg<128, 2, 128, 3, 1>>(a);
+    case 128:
+      return a.causal && a.Nk <= kCskipMaxKeys
+                 ? run_fwd<FwdCfg<128, 2, 128, 3, 1, false, false, true>>(a)
+                 : run_fwd<FwdCfg<128, 2, 128, 3, 1>>(a);
     case 256: return run_fwd<FwdCfg<256, 1, 128, 2, 1>>(a);
     default: return 2;
   }
@@ -997,12 +1029,18 @@ int launch_fwd_bf16_sm100(const AttnArgs &a) {
   switch (a.d) {
     // dropout (not in split mode) at d = 64, 128: one Q tile per CTA, with
     // warps 4-7 evaluating the mask
+    // causal, one piece, up to kCskipMaxKeys keys: the instances whose tile 0
+    // stops one block early
     case 64:
-      return a.drop_thr && a.splits == 1 ? run_fwd<FwdCfg<64, 1, 128, 4, 2, true>>(a)
-                                         : run_fwd<FwdCfg<64, 2, 128, 3, 2>>(a);
+      if (a.drop_thr && a.splits == 1) return run_fwd<FwdCfg<64, 1, 128, 4, 2, true>>(a);
+      if (a.causal && a.splits == 1 && a.Nk <= kCskipMaxKeys)
+        return run_fwd<FwdCfg<64, 2, 128, 3, 2, false, false, true>>(a);
+      return run_fwd<FwdCfg<64, 2, 128, 3, 2>>(a);
     case 128:
-      return a.drop_thr && a.splits == 1 ? run_fwd<FwdCfg<128, 1, 128, 2, 2, true>>(a)
-                                         : run_fwd<FwdCfg<128, 2, 128, 1, 2>>(a);
+      if (a.drop_thr && a.splits == 1) return run_fwd<FwdCfg<128, 1, 128, 2, 2, true>>(a);
+      if (a.causal && a.splits == 1 && a.Nk <= kCskipMaxKeys)
+        return run_fwd<FwdCfg<128, 2, 128, 1, 2, false, false, true>>(a);
+      return run_fwd<FwdCfg<128, 2, 128, 1, 2>>(a);
     case 256:
       return a.drop_thr && a.splits == 1 ? run_fwd<FwdCfg<256, 1, 128, 1, 2, true>>(a)
                                          : run_fwd<FwdCfg<256, 1, 128, 1, 2>>(a);
