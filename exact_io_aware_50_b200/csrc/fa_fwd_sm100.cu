@@ -869,12 +869,14 @@ int run_fwd(const AttnArgs &a) {
   // B200, causal B4 H16 N8192: 2.24 -> 1.87 ms, B16 N2048 0.80 -> 0.62, B64
   // N512 0.316 -> 0.283; 24 or 96 MB groups were slower; at d = 64 and 128,
   // whose units read a quarter of those bytes per query row, grouping was
-  // neutral or slower: causal B4 H16 N4096 d128 0.289 -> 0.326 ms).
+  // neutral or slower: causal B4 H16 N4096 d128 0.289 -> 0.326 ms; the
+  // dropout instance, bound by its mask warps, gained nothing either way:
+  // p = 0.1, B4 H16 N8192 3.04 -> 3.11 ms, B16 N2048 0.97 -> 0.95).
   {
     const double kv_per_head = 2.0 * a.Nk * C::D * C::ES / (double)(a.Hq / a.Hkv);
     const double kv_all = kv_per_head * a.B * a.Hq;
     p.hg = p.BH;
-    if (C::D == 256 && C::ES == 2 && a.causal && kv_all > 256.0 * 1024 * 1024) {
+    if (C::D == 256 && C::ES == 2 && !C::MW && a.causal && kv_all > 256.0 * 1024 * 1024) {
       const double hg = (48.0 * 1024 * 1024) / kv_per_head;
       p.hg = hg < 1.0 ? 1 : (hg > p.BH ? p.BH : (int)hg);
     }
